@@ -1,0 +1,224 @@
+"""CPU oracle for group-wise weight quantization (TEST INFRASTRUCTURE ONLY).
+
+Thin numpy/ctypes wrapper around ``liboracle.so`` (plain single-threaded C99,
+``wq_oracle.c``).  Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package; the product path (the
+CUDA library and its binding in ``bit_gemm_group_b200``) never does, and the
+two share no code.
+
+Arrays are numpy; 16-bit float data (bf16, fp16) travels as its uint16 bit
+pattern.  Every function returns its outputs plus the oracle status code.
+"""
+import ctypes
+import numpy as np
+
+from . import build as _build
+
+OK = 0
+ERR_ARG = -1
+ERR_NONFINITE = -5
+ERR_OVERFLOW = -7
+
+F32, BF16, F16 = 0, 1, 2
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(_build.build())
+        _declare(_lib)
+    return _lib
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+
+
+def _declare(L):
+    L.oracle_f32_to_f16.argtypes = [ctypes.c_float]
+    L.oracle_f32_to_f16.restype = ctypes.c_uint16
+    L.oracle_f16_to_f32.argtypes = [ctypes.c_uint16]
+    L.oracle_f16_to_f32.restype = ctypes.c_float
+    L.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
+    L.oracle_f32_to_bf16.restype = ctypes.c_uint16
+    L.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    L.oracle_bf16_to_f32.restype = ctypes.c_float
+    L.oracle_round_half_even.argtypes = [ctypes.c_float]
+    L.oracle_round_half_even.restype = ctypes.c_float
+    for name in ("oracle_f32_to_f16_array", "oracle_f16_to_f32_array",
+                 "oracle_f32_to_bf16_array", "oracle_bf16_to_f32_array"):
+        getattr(L, name).argtypes = [_P, _P, _I64]
+        getattr(L, name).restype = None
+    L.oracle_quantize_int4.argtypes = [_P, _INT, _I64, _I64, _INT, _INT, _P, _P, _P]
+    L.oracle_quantize_int8_rows.argtypes = [_P, _INT, _I64, _I64, _P, _P]
+    L.oracle_quant_act_i8.argtypes = [_P, _INT, _I64, _I64, _P, _P]
+    L.oracle_dequant_int4.argtypes = [_P, _P, _P, _I64, _I64, _INT, _INT, _P]
+    L.oracle_dequant_int8_rows.argtypes = [_P, _P, _I64, _I64, _P]
+    L.oracle_gemm_w4a16.argtypes = [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _INT,
+                                    _I64, _I64, _P]
+    L.oracle_gemm_w8a8_acc.argtypes = [_P, _P, _I64, _I64, _I64, _I64, _I64, _I64,
+                                       _I64, _P]
+    L.oracle_w8a8_rescale.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P]
+    for name in ("oracle_quantize_int4", "oracle_quantize_int8_rows",
+                 "oracle_quant_act_i8", "oracle_dequant_int4",
+                 "oracle_dequant_int8_rows", "oracle_gemm_w4a16",
+                 "oracle_gemm_w8a8_acc", "oracle_w8a8_rescale"):
+        getattr(L, name).restype = _INT
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _tag_and_bits(W, dtype_tag):
+    """Return (contiguous array, tag).  float32 arrays are tagged F32; uint16
+    arrays carry bf16 or fp16 bits and need an explicit tag."""
+    if W.dtype == np.float32:
+        return _c(W, np.float32), F32
+    if W.dtype == np.uint16:
+        if dtype_tag not in (BF16, F16):
+            raise ValueError("uint16 input needs dtype_tag BF16 or F16")
+        return _c(W, np.uint16), dtype_tag
+    raise TypeError(f"unsupported input dtype {W.dtype}")
+
+
+# --- conversions -------------------------------------------------------------
+
+def f32_to_f16(x):
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint16)
+    lib().oracle_f32_to_f16_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def f16_to_f32(h):
+    h = _c(h, np.uint16)
+    out = np.empty(h.shape, np.float32)
+    lib().oracle_f16_to_f32_array(_ptr(h), _ptr(out), h.size)
+    return out
+
+
+def f32_to_bf16(x):
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint16)
+    lib().oracle_f32_to_bf16_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def bf16_to_f32(b):
+    b = _c(b, np.uint16)
+    out = np.empty(b.shape, np.float32)
+    lib().oracle_bf16_to_f32_array(_ptr(b), _ptr(out), b.size)
+    return out
+
+
+def round_half_even(v: float) -> float:
+    return float(lib().oracle_round_half_even(ctypes.c_float(v)))
+
+
+# --- quantizers ----------------------------------------------------------------
+
+def quantize_int4(W, group_size=128, sym=True, dtype_tag=None):
+    """INT4 group-wise quantize + pack.  W: [N, K] float32, or uint16 bits with
+    dtype_tag BF16/F16.  Returns (codes u8 [N, K/2], scales u16 (fp16 bits)
+    [N, K/g], zeros u16 [N, K/g] or None for sym, status)."""
+    W, tag = _tag_and_bits(W, dtype_tag)
+    N, K = W.shape
+    G = K // group_size if group_size > 0 else 0
+    codes = np.zeros((N, K // 2), np.uint8)
+    scales = np.zeros((N, G), np.uint16)
+    zeros = None if sym else np.zeros((N, G), np.uint16)
+    st = lib().oracle_quantize_int4(_ptr(W), tag, N, K, group_size, int(bool(sym)),
+                                    _ptr(codes), _ptr(scales), _ptr(zeros))
+    return codes, scales, zeros, st
+
+
+def quantize_int8_rows(W, dtype_tag=None):
+    """Per-output-channel symmetric INT8.  Returns (q int8 [N, K], scales f32 [N], status)."""
+    W, tag = _tag_and_bits(W, dtype_tag)
+    N, K = W.shape
+    q = np.zeros((N, K), np.int8)
+    s = np.zeros((N,), np.float32)
+    st = lib().oracle_quantize_int8_rows(_ptr(W), tag, N, K, _ptr(q), _ptr(s))
+    return q, s, st
+
+
+def quant_act_i8(X, dtype_tag=None):
+    """Per-token dynamic INT8.  Returns (q int8 [M, K], scales f32 [M], status)."""
+    X, tag = _tag_and_bits(X, dtype_tag)
+    M, K = X.shape
+    q = np.zeros((M, K), np.int8)
+    s = np.zeros((M,), np.float32)
+    st = lib().oracle_quant_act_i8(_ptr(X), tag, M, K, _ptr(q), _ptr(s))
+    return q, s, st
+
+
+def dequant_int4(codes, scales, zeros, K, group_size=128, sym=True):
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint16)
+    zeros = None if zeros is None else _c(zeros, np.uint16)
+    N = codes.shape[0]
+    out = np.zeros((N, K), np.float32)
+    st = lib().oracle_dequant_int4(_ptr(codes), _ptr(scales), _ptr(zeros), N, K,
+                                   group_size, int(bool(sym)), _ptr(out))
+    return out, st
+
+
+def dequant_int8_rows(q, scales):
+    q = _c(q, np.int8)
+    scales = _c(scales, np.float32)
+    N, K = q.shape
+    out = np.zeros((N, K), np.float32)
+    st = lib().oracle_dequant_int8_rows(_ptr(q), _ptr(scales), N, K, _ptr(out))
+    return out, st
+
+
+# --- products --------------------------------------------------------------------
+
+def gemm_w4a16(X_bf16_bits, codes, scales, zeros, group_size=128, sym=True,
+               n0=0, n1=None):
+    """fp64 Y[:, n0:n1] = X * dequant(W)^T.  X as uint16 bf16 bits [M, K]."""
+    X = _c(X_bf16_bits, np.uint16)
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint16)
+    zeros = None if zeros is None else _c(zeros, np.uint16)
+    M, K = X.shape
+    N = codes.shape[0]
+    n1 = N if n1 is None else n1
+    Y = np.zeros((M, n1 - n0), np.float64)
+    st = lib().oracle_gemm_w4a16(_ptr(X), M, K, _ptr(codes), _ptr(scales),
+                                 _ptr(zeros), N, group_size, int(bool(sym)),
+                                 n0, n1, _ptr(Y))
+    return Y, st
+
+
+def gemm_w8a8_acc(qx, qw, m0=0, m1=None, n0=0, n1=None):
+    qx = _c(qx, np.int8)
+    qw = _c(qw, np.int8)
+    M, K = qx.shape
+    N = qw.shape[0]
+    m1 = M if m1 is None else m1
+    n1 = N if n1 is None else n1
+    acc = np.zeros((m1 - m0, n1 - n0), np.int32)
+    st = lib().oracle_gemm_w8a8_acc(_ptr(qx), _ptr(qw), M, N, K, m0, m1, n0, n1,
+                                    _ptr(acc))
+    return acc, st
+
+
+def w8a8_rescale(acc, sx, sw, m0=0, n0=0):
+    acc = _c(acc, np.int32)
+    sx = _c(sx, np.float32)
+    sw = _c(sw, np.float32)
+    m1 = m0 + acc.shape[0]
+    n1 = n0 + acc.shape[1]
+    Y = np.zeros(acc.shape, np.float64)
+    st = lib().oracle_w8a8_rescale(_ptr(acc), _ptr(sx), _ptr(sw), m0, m1, n0, n1,
+                                   _ptr(Y))
+    return Y, st

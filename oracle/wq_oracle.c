@@ -1,0 +1,436 @@
+/*
+ * wq_oracle.c -- plain, slow, single-threaded CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY: called by the tests, the smoke check and the
+ * benchmark's CPU-baseline leg; never by the product path.  Shares no code
+ * with the CUDA library.
+ *
+ * Every step follows the order in which the quantization write-ups state it;
+ * each function names the page section it restates.  Floating-point decisions
+ * that pick an integer code are taken in binary32, the same precision as the
+ * kernels; matrix products are summed in binary64.  The page tags [P1]..[P4]
+ * are listed with their titles in wq_oracle.h.
+ */
+#include "wq_oracle.h"
+
+#include <math.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------- */
+/* Rounding and format conversion (IEEE-754 definitions)                      */
+/* ------------------------------------------------------------------------- */
+
+/* Round a double that holds a non-negative value to the nearest integer,
+ * ties to the even integer.  Exact: floor() and the subtraction are exact for
+ * the magnitudes used here (< 2^52). */
+static double round_half_even_nonneg(double q) {
+  double n = floor(q);
+  double d = q - n;
+  if (d > 0.5) return n + 1.0;
+  if (d < 0.5) return n;
+  return (fmod(n, 2.0) == 0.0) ? n : n + 1.0;
+}
+
+float oracle_round_half_even(float v) {
+  /* numpy.round / torch.round round half to even ([P3] sec. 2.1 code,
+   * [P4] sec. 2.1 code); reproduce that on a binary32 value. */
+  if (!isfinite(v)) return v;
+  double a = fabs((double)v);
+  if (a >= 8388608.0) return v; /* already an integer (>= 2^23) */
+  double r = round_half_even_nonneg(a);
+  return (float)(v < 0 ? -r : r);
+}
+
+static uint32_t f32_bits(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  return u;
+}
+
+static float f32_from_bits(uint32_t u) {
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* binary32 -> binary16, round to nearest even. */
+uint16_t oracle_f32_to_f16(float f) {
+  uint16_t sign = (uint16_t)((f32_bits(f) >> 31) << 15);
+  if (isnan(f)) return (uint16_t)(sign | 0x7E00u);
+  double a = fabs((double)f);
+  /* largest finite binary16 is 65504; the midpoint to the next power of two
+   * (65520) has an odd neighbour (0x7BFF), so ties round up to infinity. */
+  if (a >= 65520.0) return (uint16_t)(sign | 0x7C00u);
+  if (a < ldexp(1.0, -14)) {
+    /* subnormal range: value = n * 2^-24, n in [0, 1024] (1024 is the
+     * smallest normal, whose encoding 0x0400 is exactly n). */
+    double n = round_half_even_nonneg(a * ldexp(1.0, 24));
+    return (uint16_t)(sign | (uint16_t)n);
+  }
+  int e;
+  double m = frexp(a, &e); /* a = m * 2^e, m in [0.5, 1) */
+  m *= 2.0;
+  e -= 1; /* a = m * 2^e, m in [1, 2) */
+  double r = round_half_even_nonneg((m - 1.0) * 1024.0);
+  if (r == 1024.0) {
+    r = 0.0;
+    e += 1;
+  }
+  if (e > 15) return (uint16_t)(sign | 0x7C00u);
+  return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)r);
+}
+
+float oracle_f16_to_f32(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1F;
+  int mant = h & 0x3FF;
+  double v;
+  if (e == 0x1F) {
+    if (mant) return NAN;
+    v = INFINITY;
+  } else if (e == 0) {
+    v = ldexp((double)mant, -24);
+  } else {
+    v = ldexp(1.0 + mant / 1024.0, e - 15);
+  }
+  return (float)(sign ? -v : v);
+}
+
+/* binary32 -> bfloat16 (1 sign, 8 exponent, 7 fraction bits), nearest even. */
+uint16_t oracle_f32_to_bf16(float f) {
+  uint16_t sign = (uint16_t)((f32_bits(f) >> 31) << 15);
+  if (isnan(f)) return (uint16_t)(sign | 0x7FC0u);
+  double a = fabs((double)f);
+  if (isinf(f)) return (uint16_t)(sign | 0x7F80u);
+  /* largest finite bfloat16 is (2 - 2^-7) * 2^127; the midpoint to 2^128 has
+   * an odd neighbour, so it rounds up to infinity */
+  if (a >= (2.0 - ldexp(1.0, -8)) * ldexp(1.0, 127))
+    return (uint16_t)(sign | 0x7F80u);
+  if (a < ldexp(1.0, -126)) {
+    double n = round_half_even_nonneg(a * ldexp(1.0, 133));
+    return (uint16_t)(sign | (uint16_t)n);
+  }
+  int e;
+  double m = frexp(a, &e);
+  m *= 2.0;
+  e -= 1;
+  double r = round_half_even_nonneg((m - 1.0) * 128.0);
+  if (r == 128.0) {
+    r = 0.0;
+    e += 1;
+  }
+  if (e > 127) return (uint16_t)(sign | 0x7F80u);
+  return (uint16_t)(sign | (uint16_t)((e + 127) << 7) | (uint16_t)r);
+}
+
+float oracle_bf16_to_f32(uint16_t b) {
+  /* bfloat16 is the top half of a binary32 pattern: widening is exact. */
+  return f32_from_bits(((uint32_t)b) << 16);
+}
+
+void oracle_f32_to_f16_array(const float *in, uint16_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_f16(in[i]);
+}
+void oracle_f16_to_f32_array(const uint16_t *in, float *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_f16_to_f32(in[i]);
+}
+void oracle_f32_to_bf16_array(const float *in, uint16_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_bf16(in[i]);
+}
+void oracle_bf16_to_f32_array(const uint16_t *in, float *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_to_f32(in[i]);
+}
+
+static float load_elem(const void *p, int dtype, int64_t i) {
+  switch (dtype) {
+    case ORACLE_F32:
+      return ((const float *)p)[i];
+    case ORACLE_BF16:
+      return oracle_bf16_to_f32(((const uint16_t *)p)[i]);
+    default:
+      return oracle_f16_to_f32(((const uint16_t *)p)[i]);
+  }
+}
+
+static int clamp_int(int v, int lo, int hi) {
+  return v < lo ? lo : (v > hi ? hi : v);
+}
+
+/* ------------------------------------------------------------------------- */
+/* INT4 group-wise quantize and pack                                          */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * For each output row n and each group of `group_size` consecutive input
+ * columns ([P4] sec. 2.2: W is [out_features, in_features], one scale per 128
+ * input dims; [P3] sec. 2.2 per-group):
+ *
+ * symmetric ([P3] sec. 2.1 symmetric_quantize, [P4] sec. 2.1):
+ *   amax = max |x|;  s = amax / (2^(b-1) - 1) = amax / 7;
+ *   q = clip(round(x / s), -8, 7);  zero point 0.
+ *   Degenerate range (amax < 1e-8): q = 0 and the returned scale is amax.
+ * asymmetric ([P3] sec. 2.1 asymmetric_quantize, [P4] sec. 2.1):
+ *   s = (max - min) / (2^b - 1) = (max - min) / 15;
+ *   z = clip(round(-min / s), 0, 15);  q = clip(round(x / s) + z, 0, 15).
+ *   Degenerate range (max - min < 1e-8): q = 0, s = 1.0, z = 0.
+ *
+ * Readings where the pages leave a step open:
+ *   - the scale is stored as fp16 ([P4] sec. 2.2 and 8 keep one fp16 scale
+ *     for every 128 INT4 weights) and the rounded, stored scale is the one the codes
+ *     are computed with, so dequantization reproduces exactly what the codes
+ *     mean; a scale that rounds to fp16 zero is treated as a degenerate range;
+ *   - round-then-add (round(x/s) + z), as in [P1] sec. 2.2, [P2] sec. 2 and
+ *     [P4] sec. 2.1; rounding is half to even as numpy/torch round;
+ *   - the fp32 division is a single IEEE division (x / s, not x * (1/s));
+ *   - storage: unsigned nibble u = q - qmin (sym: q + 8, asym: q), two per
+ *     byte, element k of row n in byte n*K/2 + k/2, low nibble = even k;
+ *     zero points are stored as fp16 integers 0..15 (asym only).
+ */
+int oracle_quantize_int4(const void *W, int w_dtype, int64_t N, int64_t K,
+                         int group_size, int sym, uint8_t *codes,
+                         uint16_t *scales, uint16_t *zeros) {
+  if (N < 0 || K < 0 || group_size <= 0 || (K % group_size) != 0 ||
+      (K % 2) != 0)
+    return ORACLE_ERR_ARG;
+  if (!sym && zeros == NULL) return ORACLE_ERR_ARG;
+  int status = ORACLE_OK;
+  const int64_t G = K / group_size;
+  const int qmin = sym ? -8 : 0;
+  const int qmax = sym ? 7 : 15;
+  memset(codes, 0, (size_t)(N * (K / 2)));
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t g = 0; g < G; ++g) {
+      const int64_t k0 = g * group_size;
+      float mn = INFINITY, mx = -INFINITY, amax = 0.0f;
+      for (int64_t k = k0; k < k0 + group_size; ++k) {
+        float x = load_elem(W, w_dtype, n * K + k);
+        if (!isfinite(x)) status = ORACLE_ERR_NONFINITE;
+        if (x < mn) mn = x;
+        if (x > mx) mx = x;
+        if (fabsf(x) > amax) amax = fabsf(x);
+      }
+      uint16_t s16;
+      int z = 0;
+      int degenerate;
+      if (sym) {
+        float s32 = amax / 7.0f;
+        s16 = oracle_f32_to_f16(s32);
+        degenerate = (amax < 1e-8f) || (oracle_f16_to_f32(s16) == 0.0f);
+        if (degenerate) s16 = oracle_f32_to_f16(amax);
+      } else {
+        float range = mx - mn;
+        float s32 = range / 15.0f;
+        s16 = oracle_f32_to_f16(s32);
+        degenerate = (range < 1e-8f) || (oracle_f16_to_f32(s16) == 0.0f);
+        if (degenerate) {
+          s16 = oracle_f32_to_f16(1.0f);
+          z = 0;
+        } else {
+          float sf = oracle_f16_to_f32(s16);
+          float zr = oracle_round_half_even(-mn / sf);
+          z = (int)fmaxf(0.0f, fminf(15.0f, zr));
+        }
+        zeros[n * G + g] = oracle_f32_to_f16((float)z);
+      }
+      if (isinf(oracle_f16_to_f32(s16))) status = ORACLE_ERR_NONFINITE;
+      scales[n * G + g] = s16;
+      const float sf = oracle_f16_to_f32(s16);
+      for (int64_t k = k0; k < k0 + group_size; ++k) {
+        int q;
+        if (degenerate) {
+          q = 0;
+        } else {
+          float x = load_elem(W, w_dtype, n * K + k);
+          float r = oracle_round_half_even(x / sf);
+          /* clamp in float first so huge quotients do not overflow int */
+          r = fmaxf(-64.0f, fminf(64.0f, r));
+          q = clamp_int((int)r + z, qmin, qmax);
+        }
+        uint8_t u = (uint8_t)(q - qmin);
+        uint8_t *byte = &codes[n * (K / 2) + k / 2];
+        if ((k & 1) == 0)
+          *byte = (uint8_t)((*byte & 0xF0u) | u);
+        else
+          *byte = (uint8_t)((*byte & 0x0Fu) | (uint8_t)(u << 4));
+      }
+    }
+  }
+  return status;
+}
+
+/* ------------------------------------------------------------------------- */
+/* INT8 symmetric rows (per-output-channel weights)                           */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * [P4] sec. 2.2: INT8 weights need only a per-channel scale -- one scale per output
+ * row; [P4] sec. 2.1 / [P3] sec. 2.1 symmetric min-max: s = amax / 127,
+ * q = clip(round(x / s)).  The clip range is [-127, 127]: [P3] sec. 2.1 maps
+ * the symmetric interval onto integers symmetric about zero.  The scale
+ * stays fp32 (it feeds the fp32 rescale of the int32 accumulator).
+ * Degenerate row (amax < 1e-8): q = 0, scale = amax ([P3] sec. 2.1).
+ */
+int oracle_quantize_int8_rows(const void *W, int w_dtype, int64_t N, int64_t K,
+                              int8_t *q, float *scales) {
+  if (N < 0 || K <= 0) return ORACLE_ERR_ARG;
+  int status = ORACLE_OK;
+  for (int64_t n = 0; n < N; ++n) {
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+      float x = load_elem(W, w_dtype, n * K + k);
+      if (!isfinite(x)) status = ORACLE_ERR_NONFINITE;
+      if (fabsf(x) > amax) amax = fabsf(x);
+    }
+    int degenerate = amax < 1e-8f;
+    float s = degenerate ? amax : amax / 127.0f;
+    scales[n] = s;
+    for (int64_t k = 0; k < K; ++k) {
+      int v = 0;
+      if (!degenerate) {
+        float r = oracle_round_half_even(load_elem(W, w_dtype, n * K + k) / s);
+        r = fmaxf(-200.0f, fminf(200.0f, r));
+        v = clamp_int((int)r, -127, 127);
+      }
+      q[n * K + k] = (int8_t)v;
+    }
+  }
+  return status;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Per-token dynamic INT8 activations                                         */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * [P4] sec. 6 (quant_kv_per_token, the per-token absmax quantizer; W8A8 uses
+ * it for activation rows, [P4] sec. 2.3):
+ *   scale = amax(|v|) / 127;  scale = max(scale, 1e-8);
+ *   q = clamp(round(v / scale), -128, 127).
+ */
+int oracle_quant_act_i8(const void *X, int x_dtype, int64_t M, int64_t K,
+                        int8_t *q, float *scales) {
+  if (M < 0 || K <= 0) return ORACLE_ERR_ARG;
+  int status = ORACLE_OK;
+  for (int64_t m = 0; m < M; ++m) {
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+      float x = load_elem(X, x_dtype, m * K + k);
+      if (!isfinite(x)) status = ORACLE_ERR_NONFINITE;
+      if (fabsf(x) > amax) amax = fabsf(x);
+    }
+    float s = amax / 127.0f;
+    if (s < 1e-8f) s = 1e-8f;
+    scales[m] = s;
+    for (int64_t k = 0; k < K; ++k) {
+      float r = oracle_round_half_even(load_elem(X, x_dtype, m * K + k) / s);
+      r = fmaxf(-200.0f, fminf(200.0f, r));
+      q[m * K + k] = (int8_t)clamp_int((int)r, -128, 127);
+    }
+  }
+  return status;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Dequantization                                                             */
+/* ------------------------------------------------------------------------- */
+
+/* [P2] sec. 2: f' = S * (q - Z); [P4] sec. 2.1: x_hat = s * (q - z).
+ * With the stored unsigned nibble u = q - qmin this is s * (u - z_eff) with
+ * z_eff = 8 (symmetric, q = u - 8, Z = 0) or z_eff = z (asymmetric, q = u).
+ * The fp16 scale has 11 significant bits and |u - z_eff| <= 15, so the
+ * binary32 product is exact. */
+int oracle_dequant_int4(const uint8_t *codes, const uint16_t *scales,
+                        const uint16_t *zeros, int64_t N, int64_t K,
+                        int group_size, int sym, float *out) {
+  if (group_size <= 0 || (K % group_size) != 0 || (K % 2) != 0)
+    return ORACLE_ERR_ARG;
+  if (!sym && zeros == NULL) return ORACLE_ERR_ARG;
+  const int64_t G = K / group_size;
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) {
+      uint8_t byte = codes[n * (K / 2) + k / 2];
+      int u = (k & 1) ? (byte >> 4) : (byte & 0x0F);
+      int64_t g = k / group_size;
+      float s = oracle_f16_to_f32(scales[n * G + g]);
+      int zeff = sym ? 8 : (int)oracle_f16_to_f32(zeros[n * G + g]);
+      out[n * K + k] = s * (float)(u - zeff);
+    }
+  }
+  return ORACLE_OK;
+}
+
+int oracle_dequant_int8_rows(const int8_t *q, const float *scales, int64_t N,
+                             int64_t K, float *out) {
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k)
+      out[n * K + k] = scales[n] * (float)q[n * K + k];
+  return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Matrix products                                                            */
+/* ------------------------------------------------------------------------- */
+
+/* W4A16 ([P4] sec. 2.3: INT4 weights, 16-bit activations, the weight is
+ * dequantized before the product): Y = X * dequant(W)^T, summed in fp64
+ * over k = 0 .. K-1 in order. */
+int oracle_gemm_w4a16(const uint16_t *X, int64_t M, int64_t K,
+                      const uint8_t *codes, const uint16_t *scales,
+                      const uint16_t *zeros, int64_t N, int group_size,
+                      int sym, int64_t n0, int64_t n1, double *Y) {
+  if (n0 < 0 || n1 > N || n0 > n1 || group_size <= 0 ||
+      (K % group_size) != 0 || (K % 2) != 0)
+    return ORACLE_ERR_ARG;
+  if (!sym && zeros == NULL) return ORACLE_ERR_ARG;
+  const int64_t G = K / group_size;
+  const int64_t W = n1 - n0;
+  for (int64_t n = n0; n < n1; ++n) {
+    for (int64_t m = 0; m < M; ++m) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        uint8_t byte = codes[n * (K / 2) + k / 2];
+        int u = (k & 1) ? (byte >> 4) : (byte & 0x0F);
+        int64_t g = k / group_size;
+        float s = oracle_f16_to_f32(scales[n * G + g]);
+        int zeff = sym ? 8 : (int)oracle_f16_to_f32(zeros[n * G + g]);
+        double w = (double)(s * (float)(u - zeff));
+        acc += (double)oracle_bf16_to_f32(X[m * K + k]) * w;
+      }
+      Y[m * W + (n - n0)] = acc;
+    }
+  }
+  return ORACLE_OK;
+}
+
+/* W8A8 ([P4] sec. 2.3 and 4.2: int8 x int8 on the integer tensor core):
+ * exact integer sums, checked to fit the int32 accumulator. */
+int oracle_gemm_w8a8_acc(const int8_t *qx, const int8_t *qw, int64_t M,
+                         int64_t N, int64_t K, int64_t m0, int64_t m1,
+                         int64_t n0, int64_t n1, int32_t *acc) {
+  if (m0 < 0 || m1 > M || m0 > m1 || n0 < 0 || n1 > N || n0 > n1)
+    return ORACLE_ERR_ARG;
+  int status = ORACLE_OK;
+  const int64_t W = n1 - n0;
+  for (int64_t m = m0; m < m1; ++m) {
+    for (int64_t n = n0; n < n1; ++n) {
+      int64_t s = 0;
+      for (int64_t k = 0; k < K; ++k)
+        s += (int64_t)qx[m * K + k] * (int64_t)qw[n * K + k];
+      if (s > INT32_MAX || s < INT32_MIN) status = ORACLE_ERR_OVERFLOW;
+      acc[(m - m0) * W + (n - n0)] = (int32_t)s;
+    }
+  }
+  return status;
+}
+
+/* Rescale of the integer accumulator by the two per-row scales, in fp64. */
+int oracle_w8a8_rescale(const int32_t *acc, const float *sx, const float *sw,
+                        int64_t m0, int64_t m1, int64_t n0, int64_t n1,
+                        double *Y) {
+  const int64_t W = n1 - n0;
+  for (int64_t m = m0; m < m1; ++m)
+    for (int64_t n = n0; n < n1; ++n)
+      Y[(m - m0) * W + (n - n0)] = (double)acc[(m - m0) * W + (n - n0)] *
+                                   (double)sx[m] * (double)sw[n];
+  return ORACLE_OK;
+}

@@ -1,0 +1,96 @@
+/*
+ * wq_oracle.h -- CPU oracle for group-wise affine weight quantization and the
+ * W4A16 / W8A8 matrix products.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the CUDA library and
+ * its Python binding) includes, links or calls this code; only the tests, the
+ * smoke check and the benchmark's CPU-baseline leg do.  It shares no code with
+ * the CUDA sources.
+ *
+ * Plain single-threaded C99, compiled with -O2 -ffp-contract=off and no
+ * fast-math, so every float operation below is one IEEE-754 binary32 (or
+ * binary64) operation rounded to nearest-even.
+ *
+ * Sources (page titles from the quantization write-ups this library follows):
+ *   [P1] "大模型量化技术入门：为什么我们需要量化？" sec. 2.2 (linear quantization formula)
+ *   [P2] "从0到1：大模型量化" sec. 2 (q = round(f/S) + Z, f' = S(q - Z))
+ *   [P3] "从 FP32 到 INT4：大模型推理加速中的量化优化实战路径" sec. 2.1 (symmetric /
+ *        asymmetric quantizers with their degenerate-range rules), sec. 2.2
+ *        (per-group granularity), sec. 4 (metadata share)
+ *   [P4] "27届大模型面试准备（十九）：模型量化全攻略" sec. 2.1 (affine quantization,
+ *        min-max scale), 2.2 (per-group g=128, 4.25-bit), 3 (per-tensor worked
+ *        example), 6 (per-token absmax quantizer)
+ *
+ * Status codes returned by the oracle functions.
+ */
+#ifndef WQ_ORACLE_H
+#define WQ_ORACLE_H
+#include <stdint.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG (-1)
+#define ORACLE_ERR_NONFINITE (-5)
+#define ORACLE_ERR_OVERFLOW (-7)
+
+/* element type tags for raw input buffers */
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+#define ORACLE_F16 2
+
+/* IEEE-754 conversions written from the format definitions (round to nearest,
+ * ties to even).  f16 = binary16 (1/5/10), bf16 = 1/8/7. */
+uint16_t oracle_f32_to_f16(float f);
+float oracle_f16_to_f32(uint16_t h);
+uint16_t oracle_f32_to_bf16(float f);
+float oracle_bf16_to_f32(uint16_t b);
+/* element-wise array forms of the four conversions */
+void oracle_f32_to_f16_array(const float *in, uint16_t *out, int64_t n);
+void oracle_f16_to_f32_array(const uint16_t *in, float *out, int64_t n);
+void oracle_f32_to_bf16_array(const float *in, uint16_t *out, int64_t n);
+void oracle_bf16_to_f32_array(const uint16_t *in, float *out, int64_t n);
+/* round-half-to-even of a float to an integer-valued float */
+float oracle_round_half_even(float v);
+
+/* INT4 group-wise quantize + pack ([P4] sec. 2.1-2.2, [P3] sec. 2.1). */
+int oracle_quantize_int4(const void *W, int w_dtype, int64_t N, int64_t K,
+                         int group_size, int sym, uint8_t *codes,
+                         uint16_t *scales, uint16_t *zeros);
+
+/* INT8 symmetric quantization with one fp32 scale per row of K elements.
+ * Used for per-output-channel weights ([P4] sec. 2.2) with qmin = -127. */
+int oracle_quantize_int8_rows(const void *W, int w_dtype, int64_t N, int64_t K,
+                              int8_t *q, float *scales);
+
+/* Per-token dynamic INT8 activation quantization ([P4] sec. 6). */
+int oracle_quant_act_i8(const void *X, int x_dtype, int64_t M, int64_t K,
+                        int8_t *q, float *scales);
+
+/* Dequantize INT4 codes to fp32: x_hat = s * (u - z_eff) ([P2] sec. 2). */
+int oracle_dequant_int4(const uint8_t *codes, const uint16_t *scales,
+                        const uint16_t *zeros, int64_t N, int64_t K,
+                        int group_size, int sym, float *out);
+
+/* Dequantize INT8 per-row codes to fp32: x_hat = s * q. */
+int oracle_dequant_int8_rows(const int8_t *q, const float *scales, int64_t N,
+                             int64_t K, float *out);
+
+/* W4A16 product in fp64: Y[m, n - n0] = sum_k X[m,k] * x_hat[n,k] for
+ * n in [n0, n1).  X is bf16 [M, K] row-major; Y is [M, n1 - n0]. */
+int oracle_gemm_w4a16(const uint16_t *X, int64_t M, int64_t K,
+                      const uint8_t *codes, const uint16_t *scales,
+                      const uint16_t *zeros, int64_t N, int group_size,
+                      int sym, int64_t n0, int64_t n1, double *Y);
+
+/* W8A8 exact integer accumulators: acc[m - m0, n - n0] = sum_k qx[m,k]*qw[n,k]
+ * for m in [m0, m1), n in [n0, n1).  Returns ORACLE_ERR_OVERFLOW if a sum
+ * does not fit int32. */
+int oracle_gemm_w8a8_acc(const int8_t *qx, const int8_t *qw, int64_t M,
+                         int64_t N, int64_t K, int64_t m0, int64_t m1,
+                         int64_t n0, int64_t n1, int32_t *acc);
+
+/* W8A8 rescale in fp64: Y = acc * sx[m] * sw[n] over the same window. */
+int oracle_w8a8_rescale(const int32_t *acc, const float *sx, const float *sw,
+                        int64_t m0, int64_t m1, int64_t n0, int64_t n1,
+                        double *Y);
+
+#endif
