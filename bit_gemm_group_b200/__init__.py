@@ -1,0 +1,238 @@
+"""bit_gemm_group_b200 -- Python binding of libwq (include/wq.h).
+
+Group-wise affine weight quantization and fused-dequantize W4A16 / W8A8 matrix
+products for NVIDIA B200 (sm_100a).  This module only marshals arguments:
+each function with a ``wq_`` name calls the C entry point of the same name
+with the tensors' device pointers and the current CUDA stream; every step runs
+in the library's CUDA kernels.  There is no CPU fallback: importing works
+without a GPU, but every call needs ``libwq.so`` (built by ``build()``) and an
+sm_100 device, and raises ``WQError`` otherwise.
+
+The helpers without the prefix (``quantize_pack``, ``dequant``, ``gemm_w4a16``,
+``quant_act_i8``, ``gemm_w8a8``) allocate the outputs with torch and call the
+``wq_`` functions.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwq.so")
+
+WQ_OK = 0
+WQ_ERR_ARG = -1
+WQ_ERR_UNSUPPORTED = -2
+WQ_ERR_ALIGN = -3
+WQ_ERR_CUDA = -4
+WQ_ERR_NONFINITE = -5
+WQ_ERR_TIMEOUT = -6
+WQ_ERR_WORKSPACE = -8
+WQ_ERR_NO_DEVICE = -9
+
+WQ_F32, WQ_BF16, WQ_F16 = 0, 1, 2
+
+# every symbol include/wq.h declares
+EXPORTED = (
+    "wq_quantize_pack", "wq_dequant", "wq_gemm_w4a16", "wq_quant_act_i8",
+    "wq_w8a8_workspace_bytes", "wq_gemm_w8a8", "wq_get_device_status",
+    "wq_status_str", "wq_last_cuda_error",
+)
+
+
+class WQError(RuntimeError):
+    def __init__(self, status, where=""):
+        self.status = status
+        name = _status_name(status)
+        detail = ""
+        if status == WQ_ERR_CUDA and _lib is not None:
+            detail = ": " + _lib.wq_last_cuda_error().decode()
+        super().__init__(f"{where} -> {name}{detail}")
+
+
+_lib = None
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile libwq.so in-tree (nvcc, sm_100a)."""
+    from . import _compile as _b
+    return _b.build(force=force, verbose=verbose)
+
+
+def lib():
+    """Load libwq.so once; raise loudly if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise WQError(WQ_ERR_NO_DEVICE,
+                          f"libwq.so missing at {LIB_PATH}; run bit_gemm_group_b200.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        _declare(L)
+        _lib = L
+    return _lib
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+
+def _declare(L):
+    L.wq_quantize_pack.argtypes = [_P, _INT, _I64, _I64, _INT, _INT, _INT, _P, _P, _P, _P]
+    L.wq_dequant.argtypes = [_P, _P, _P, _I64, _I64, _INT, _INT, _INT, _P, _INT, _P]
+    L.wq_gemm_w4a16.argtypes = [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _INT, _P, _P]
+    L.wq_quant_act_i8.argtypes = [_P, _I64, _I64, _P, _P, _P]
+    L.wq_w8a8_workspace_bytes.argtypes = [_I64, _I64]
+    L.wq_w8a8_workspace_bytes.restype = _SZ
+    L.wq_gemm_w8a8.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P, _P, _SZ, _P, _P]
+    L.wq_get_device_status.argtypes = [_P, _INT]
+    L.wq_status_str.argtypes = [_INT]
+    L.wq_status_str.restype = ctypes.c_char_p
+    L.wq_last_cuda_error.argtypes = []
+    L.wq_last_cuda_error.restype = ctypes.c_char_p
+    for name in ("wq_quantize_pack", "wq_dequant", "wq_gemm_w4a16", "wq_quant_act_i8",
+                 "wq_gemm_w8a8", "wq_get_device_status"):
+        getattr(L, name).restype = _INT
+
+
+def _status_name(status):
+    if _lib is not None:
+        return _lib.wq_status_str(status).decode()
+    return str(status)
+
+
+def _check(status, where):
+    if status != WQ_OK:
+        raise WQError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise WQError(WQ_ERR_ARG, "tensor is not on a CUDA device (no CPU fallback)")
+    if not t.is_contiguous():
+        raise WQError(WQ_ERR_ARG, "tensor must be contiguous (row-major)")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+_DTYPE_TAG = {torch.float32: WQ_F32, torch.bfloat16: WQ_BF16, torch.float16: WQ_F16}
+
+
+# ---------------------------------------------------------------- C-named calls
+
+def wq_quantize_pack(W, group_size, bits, sym, codes, scales, zeros=None, stream=None):
+    N, K = W.shape
+    st = lib().wq_quantize_pack(_ptr(W), _DTYPE_TAG.get(W.dtype, -1), N, K, group_size, bits,
+                                int(bool(sym)), _ptr(codes), _ptr(scales), _ptr(zeros),
+                                _stream(stream))
+    _check(st, "wq_quantize_pack")
+
+
+def wq_dequant(codes, scales, zeros, N, K, group_size, bits, sym, out, stream=None):
+    tag = _DTYPE_TAG.get(out.dtype, -1)
+    st = lib().wq_dequant(_ptr(codes), _ptr(scales), _ptr(zeros), N, K, group_size, bits,
+                          int(bool(sym)), _ptr(out), tag, _stream(stream))
+    _check(st, "wq_dequant")
+
+
+def wq_gemm_w4a16(X, codes, scales, zeros, N, group_size, sym, Y, stream=None):
+    M, K = X.shape
+    st = lib().wq_gemm_w4a16(_ptr(X), M, K, _ptr(codes), _ptr(scales), _ptr(zeros), N,
+                             group_size, int(bool(sym)), _ptr(Y), _stream(stream))
+    _check(st, "wq_gemm_w4a16")
+
+
+def wq_quant_act_i8(X, q, s, stream=None):
+    M, K = X.shape
+    st = lib().wq_quant_act_i8(_ptr(X), M, K, _ptr(q), _ptr(s), _stream(stream))
+    _check(st, "wq_quant_act_i8")
+
+
+def wq_w8a8_workspace_bytes(M, K):
+    return int(lib().wq_w8a8_workspace_bytes(M, K))
+
+
+def wq_gemm_w8a8(X, Wq, w_scales, Y, ws, acc_out=None, stream=None):
+    M, K = X.shape
+    N = Wq.shape[0]
+    st = lib().wq_gemm_w8a8(_ptr(X), M, K, _ptr(Wq), _ptr(w_scales), N, _ptr(Y), _ptr(ws),
+                            ws.numel() * ws.element_size(), _ptr(acc_out), _stream(stream))
+    _check(st, "wq_gemm_w8a8")
+
+
+def wq_get_device_status(reset=True, stream=None):
+    """Synchronize the stream and return the first kernel-detected error code."""
+    return int(lib().wq_get_device_status(_stream(stream), int(bool(reset))))
+
+
+def wq_status_str(status):
+    return lib().wq_status_str(status).decode()
+
+
+def wq_last_cuda_error():
+    return lib().wq_last_cuda_error().decode()
+
+
+# ----------------------------------------------------------- allocating helpers
+
+def quantize_pack(W, group_size=128, bits=4, sym=True):
+    """Returns (codes, scales, zeros).  bits=4: codes uint8 [N, K/2], fp16
+    scales/zeros [N, K/g] (zeros None if sym).  bits=8: int8 [N, K], fp32 [N]."""
+    N, K = W.shape
+    dev = W.device
+    if bits == 4:
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((N, K // group_size), dtype=torch.float16, device=dev)
+        zeros = None if sym else torch.empty_like(scales)
+    else:
+        codes = torch.empty((N, K), dtype=torch.int8, device=dev)
+        scales = torch.empty((N,), dtype=torch.float32, device=dev)
+        zeros = None
+        group_size = K
+    wq_quantize_pack(W, group_size, bits, sym, codes, scales, zeros)
+    return codes, scales, zeros
+
+
+def dequant(codes, scales, zeros, K, group_size=128, bits=4, sym=True,
+            out_dtype=torch.float32):
+    N = codes.shape[0]
+    out = torch.empty((N, K), dtype=out_dtype, device=codes.device)
+    wq_dequant(codes, scales, zeros, N, K, K if bits == 8 else group_size, bits, sym, out)
+    return out
+
+
+def gemm_w4a16(X, codes, scales, zeros, group_size=128, sym=True):
+    M = X.shape[0]
+    N = codes.shape[0]
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    wq_gemm_w4a16(X, codes, scales, zeros, N, group_size, sym, Y)
+    return Y
+
+
+def quant_act_i8(X):
+    M, K = X.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    s = torch.empty((M,), dtype=torch.float32, device=X.device)
+    wq_quant_act_i8(X, q, s)
+    return q, s
+
+
+def gemm_w8a8(X, Wq, w_scales, want_acc=False):
+    M, K = X.shape
+    N = Wq.shape[0]
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    ws = torch.empty((max(1, wq_w8a8_workspace_bytes(M, K)),), dtype=torch.uint8,
+                     device=X.device)
+    acc = torch.empty((M, N), dtype=torch.int32, device=X.device) if want_acc else None
+    wq_gemm_w8a8(X, Wq, w_scales, Y, ws, acc)
+    return (Y, acc) if want_acc else Y

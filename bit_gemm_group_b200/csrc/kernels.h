@@ -1,0 +1,23 @@
+// kernels.h -- internal launchers behind the C ABI (not part of the public API).
+// Each launcher assumes its arguments were validated by wq_api.cu and returns
+// a wq_status.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace wq_host {
+
+int launch_quantize_int4(const void* W, int w_dtype, int64_t N, int64_t K, int group_size,
+                         int sym, void* codes, void* scales, void* zeros, cudaStream_t s);
+int launch_quantize_rows_i8(const void* W, int w_dtype, int64_t N, int64_t K, bool activation,
+                            void* q, void* scales, cudaStream_t s);
+int launch_dequant_int4(const void* codes, const void* scales, const void* zeros, int64_t N,
+                        int64_t K, int group_size, int sym, void* out, int out_dtype,
+                        cudaStream_t s);
+int launch_dequant_int8_rows(const void* q, const void* scales, int64_t N, int64_t K, void* out,
+                             int out_dtype, cudaStream_t s);
+int launch_gemv_w4a16(const void* X, int64_t M, int64_t K, const void* codes,
+                      const void* scales, const void* zeros, int64_t N, int sym, void* Y,
+                      cudaStream_t s);
+
+}  // namespace wq_host

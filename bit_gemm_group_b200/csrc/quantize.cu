@@ -1,0 +1,420 @@
+// quantize.cu -- the memory-bound kernels of the path:
+//   * INT4 group-wise quantize + pack        ("大模型面试准备（十九）…" sec. 2.1-2.2;
+//                                             "从 FP32 到 INT4 …" sec. 2.1 quantizers)
+//   * INT8 per-row quantize (weights per output channel, activations per token;
+//                                             "大模型面试准备（十九）…" sec. 2.2, sec. 6)
+//   * dequantize x_hat = s * (q - z)         ("从0到1：大模型量化" sec. 2)
+//
+// All of them stream their input once with 16-byte (or element-sized when
+// smaller) vector loads, keep several groups in flight per warp, and size the
+// grid as a multiple of the SM count.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace wq {
+
+template <int BYTES>
+struct Vec;
+template <>
+struct Vec<16> { using type = uint4; };
+template <>
+struct Vec<8> { using type = uint2; };
+template <>
+struct Vec<4> { using type = uint32_t; };
+template <>
+struct Vec<2> { using type = uint16_t; };
+template <>
+struct Vec<1> { using type = uint8_t; };
+
+// E contiguous elements of T, loaded with the widest aligned vectors
+// (read-only, streaming: the weight is read exactly once).
+template <typename T, int E>
+struct Elems {
+  static constexpr int BYTES = E * int(sizeof(T));
+  static constexpr int V = BYTES >= 16 ? 16 : BYTES;
+  static constexpr int NV = BYTES / V;
+  using VT = typename Vec<V>::type;
+  union {
+    VT v[NV];
+    T e[E];
+  } u;
+  __device__ __forceinline__ void load(const T* p) {
+    const VT* src = reinterpret_cast<const VT*>(p);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) u.v[i] = __ldcs(src + i);
+  }
+};
+
+// ---------------------------------------------------------------------------
+// INT4 group-wise quantize + pack
+// ---------------------------------------------------------------------------
+// One warp handles one group of 32*E consecutive elements of a row (lane l owns
+// elements [l*E, l*E+E)); U groups per warp iteration are loaded before any is
+// processed, so each warp keeps U*32*E*sizeof(T) bytes in flight.  Group i of
+// the flattened [N, K/gs] grid starts at element i*gs because gs divides K.
+template <typename T, int E, int U>
+__global__ void __launch_bounds__(256) quantize_int4_kernel(
+    const T* __restrict__ W, int64_t total_groups, int sym, uint8_t* __restrict__ codes,
+    __half* __restrict__ scales, __half* __restrict__ zeros, int* status) {
+  constexpr int GS = 32 * E;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  const int qmin = sym ? -8 : 0;
+  const int qmax = sym ? 7 : 15;
+
+  for (int64_t base = warp * U; base < total_groups; base += nwarps * U) {
+    Elems<T, E> in[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j)
+      if (base + j < total_groups) in[j].load(W + (base + j) * GS + lane * E);
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int64_t gi = base + j;
+      if (gi >= total_groups) break;  // warp-uniform
+      float x[E];
+      float mn = INFINITY, mx = -INFINITY, amax = 0.f;
+      bool finite = true;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        x[e] = to_f32<T>(in[j].u.e[e]);
+        finite &= isfinite(x[e]);
+        mn = fminf(mn, x[e]);
+        mx = fmaxf(mx, x[e]);
+        amax = fmaxf(amax, fabsf(x[e]));
+      }
+      unsigned short s_bits;
+      float sf;
+      int z = 0;
+      bool degenerate;
+      if (sym) {
+        amax = warp_max(amax);
+        sf = f16_round_trip(div_rn(amax, 7.f), &s_bits);
+        degenerate = (amax < 1e-8f) || (sf == 0.f);
+        if (degenerate) sf = f16_round_trip(amax, &s_bits);
+      } else {
+        mn = warp_min(mn);
+        mx = warp_max(mx);
+        const float range = mx - mn;
+        sf = f16_round_trip(div_rn(range, 15.f), &s_bits);
+        degenerate = (range < 1e-8f) || (sf == 0.f);
+        if (degenerate) {
+          sf = f16_round_trip(1.f, &s_bits);
+        } else {
+          const float zr = round_even(div_rn(-mn, sf));
+          z = int(fmaxf(0.f, fminf(15.f, zr)));
+        }
+      }
+      finite = __all_sync(0xffffffffu, finite);
+      if (lane == 0) {
+        if (!finite || isinf(sf)) record_error(status, WQ_ERR_NONFINITE);
+        scales[gi] = __ushort_as_half(s_bits);
+        if (!sym) zeros[gi] = __int2half_rn(z);
+      }
+      // quantize + pack: E nibbles per lane, low nibble = even element
+      uint32_t nib[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        int q = 0;
+        if (!degenerate) {
+          float r = round_even(div_rn(x[e], sf));
+          r = fmaxf(-64.f, fminf(64.f, r));
+          q = min(max(int(r) + z, qmin), qmax);
+        }
+        nib[e] = uint32_t(q - qmin);
+      }
+      uint8_t* dst = codes + gi * (GS / 2);
+      if constexpr (E == 1) {
+        const uint32_t other = __shfl_down_sync(0xffffffffu, nib[0], 1);
+        if ((lane & 1) == 0) dst[lane >> 1] = uint8_t(nib[0] | (other << 4));
+      } else {
+        constexpr int NB = E / 2;  // bytes per lane
+        union {
+          typename Vec<(NB >= 16 ? 16 : NB)>::type v[(NB >= 16 ? NB / 16 : 1)];
+          uint8_t b[NB];
+        } out;
+#pragma unroll
+        for (int i = 0; i < NB; ++i) out.b[i] = uint8_t(nib[2 * i] | (nib[2 * i + 1] << 4));
+        constexpr int V = NB >= 16 ? 16 : NB;
+        using VT = typename Vec<V>::type;
+        VT* d = reinterpret_cast<VT*>(dst + lane * NB);
+#pragma unroll
+        for (int i = 0; i < NB / V; ++i) d[i] = out.v[i];
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// INT8 per-row quantization (weights per output channel / activations per token)
+// ---------------------------------------------------------------------------
+// One 256-thread block per row: pass 1 reduces amax with 16-byte loads, pass 2
+// re-reads the row (L1/L2 resident: a row is at most a few tens of KB) and
+// writes int8 codes 8 at a time.
+template <typename T, bool ACT>
+__global__ void __launch_bounds__(256) quantize_rows_i8_kernel(
+    const T* __restrict__ X, int64_t rows, int64_t K, int8_t* __restrict__ q,
+    float* __restrict__ scales, int* status) {
+  constexpr int EV = 8;  // elements per vector step
+  __shared__ float red[8];
+  __shared__ int bad_any;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const T* row = X + r * K;
+    float amax = 0.f;
+    bool finite = true;
+    for (int64_t k = int64_t(threadIdx.x) * EV; k < K; k += int64_t(blockDim.x) * EV) {
+      Elems<T, EV> v;
+      v.load(row + k);
+#pragma unroll
+      for (int e = 0; e < EV; ++e) {
+        const float x = to_f32<T>(v.u.e[e]);
+        finite &= isfinite(x);
+        amax = fmaxf(amax, fabsf(x));
+      }
+    }
+    amax = warp_max(amax);
+    const int nbad = __syncthreads_or(!finite);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float m = red[0];
+      for (int w = 1; w < int(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+      red[0] = m;
+      bad_any = nbad;
+    }
+    __syncthreads();
+    amax = red[0];
+    float s;
+    bool degenerate = false;
+    if (ACT) {
+      s = fmaxf(div_rn(amax, 127.f), 1e-8f);
+    } else {
+      degenerate = amax < 1e-8f;
+      s = degenerate ? amax : div_rn(amax, 127.f);
+    }
+    if (threadIdx.x == 0) {
+      scales[r] = s;
+      if (bad_any) record_error(status, WQ_ERR_NONFINITE);
+    }
+    const int lo = ACT ? -128 : -127;
+    for (int64_t k = int64_t(threadIdx.x) * EV; k < K; k += int64_t(blockDim.x) * EV) {
+      Elems<T, EV> v;
+      v.load(row + k);
+      union {
+        uint2 v2;
+        int8_t b[EV];
+      } o;
+#pragma unroll
+      for (int e = 0; e < EV; ++e) {
+        int qi = 0;
+        if (!degenerate) {
+          float rr = round_even(div_rn(to_f32<T>(v.u.e[e]), s));
+          rr = fmaxf(-200.f, fminf(200.f, rr));
+          qi = min(max(int(rr), lo), 127);
+        }
+        o.b[e] = int8_t(qi);
+      }
+      *reinterpret_cast<uint2*>(q + r * K + k) = o.v2;
+    }
+    __syncthreads();  // red[] is reused by the next row
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Dequantization
+// ---------------------------------------------------------------------------
+// One thread expands 16 bytes of codes (32 elements) of one row.
+template <typename OutT>
+__global__ void __launch_bounds__(256) dequant_int4_kernel(
+    const uint8_t* __restrict__ codes, const __half* __restrict__ scales,
+    const __half* __restrict__ zeros, int64_t N, int64_t K, int gs, int sym,
+    OutT* __restrict__ out) {
+  const int64_t chunks_per_row = K / 32;
+  const int64_t total = N * chunks_per_row;
+  const int64_t G = K / gs;
+  for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < total;
+       c += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t n = c / chunks_per_row;
+    const int64_t k0 = (c % chunks_per_row) * 32;
+    const uint4 w = __ldcs(reinterpret_cast<const uint4*>(codes + n * (K / 2) + k0 / 2));
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    float vals[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int64_t k = k0 + i;
+      const int64_t g = k / gs;  // gs >= 32 and 32 | gs: at most one change per chunk
+      const float s = __half2float(scales[n * G + g]);
+      const int zeff = sym ? 8 : int(__half2float(zeros[n * G + g]));
+      const int u = int((words[i >> 3] >> (4 * (i & 7))) & 0xFu);
+      vals[i] = s * float(u - zeff);  // exact: 11-bit scale times |u - z| <= 15
+    }
+    OutT* dst = out + n * K + k0;
+    if constexpr (sizeof(OutT) == 4) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        __stcs(reinterpret_cast<float4*>(dst) + i,
+               make_float4(vals[4 * i], vals[4 * i + 1], vals[4 * i + 2], vals[4 * i + 3]));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        union {
+          uint4 v;
+          __nv_bfloat162 h[4];
+        } o;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          o.h[j] = __floats2bfloat162_rn(vals[8 * i + 2 * j], vals[8 * i + 2 * j + 1]);
+        __stcs(reinterpret_cast<uint4*>(dst) + i, o.v);
+      }
+    }
+  }
+}
+
+template <typename OutT>
+__global__ void __launch_bounds__(256) dequant_int8_rows_kernel(
+    const int8_t* __restrict__ q, const float* __restrict__ scales, int64_t N, int64_t K,
+    OutT* __restrict__ out) {
+  const int64_t chunks_per_row = K / 16;
+  const int64_t total = N * chunks_per_row;
+  for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < total;
+       c += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t n = c / chunks_per_row;
+    const int64_t k0 = (c % chunks_per_row) * 16;
+    union {
+      uint4 v;
+      int8_t b[16];
+    } w;
+    w.v = __ldcs(reinterpret_cast<const uint4*>(q + n * K + k0));
+    const float s = scales[n];
+    OutT* dst = out + n * K + k0;
+    if constexpr (sizeof(OutT) == 4) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        __stcs(reinterpret_cast<float4*>(dst) + i,
+               make_float4(s * w.b[4 * i], s * w.b[4 * i + 1], s * w.b[4 * i + 2],
+                           s * w.b[4 * i + 3]));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        union {
+          uint4 v;
+          __nv_bfloat162 h[4];
+        } o;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          o.h[j] = __floats2bfloat162_rn(s * w.b[8 * i + 2 * j], s * w.b[8 * i + 2 * j + 1]);
+        __stcs(reinterpret_cast<uint4*>(dst) + i, o.v);
+      }
+    }
+  }
+}
+
+}  // namespace wq
+
+// ---------------------------------------------------------------------------
+// Launchers
+// ---------------------------------------------------------------------------
+namespace wq_host {
+
+static int grid_for(int64_t work_items, int items_per_block) {
+  const int64_t blocks = (work_items + items_per_block - 1) / items_per_block;
+  const int64_t cap = int64_t(sm_count()) * 8;  // 8 resident 256-thread blocks per SM
+  return int(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
+}
+
+template <typename T, int E>
+static void quantize_int4_typed(const void* W, int64_t N, int64_t K, int sym, void* codes,
+                                void* scales, void* zeros, cudaStream_t s) {
+  constexpr int U = E >= 8 ? 2 : 4;
+  const int64_t total = N * (K / (32 * E));
+  const int64_t warps = (total + U - 1) / U;
+  wq::quantize_int4_kernel<T, E, U><<<grid_for(warps, 8), 256, 0, s>>>(
+      static_cast<const T*>(W), total, sym, static_cast<uint8_t*>(codes),
+      static_cast<__half*>(scales), static_cast<__half*>(zeros), status_ptr());
+}
+
+template <typename T>
+static int quantize_int4_dispatch(const void* W, int64_t N, int64_t K, int gs, int sym,
+                                  void* codes, void* scales, void* zeros, cudaStream_t s) {
+  switch (gs) {
+    case 32: quantize_int4_typed<T, 1>(W, N, K, sym, codes, scales, zeros, s); break;
+    case 64: quantize_int4_typed<T, 2>(W, N, K, sym, codes, scales, zeros, s); break;
+    case 128: quantize_int4_typed<T, 4>(W, N, K, sym, codes, scales, zeros, s); break;
+    case 256: quantize_int4_typed<T, 8>(W, N, K, sym, codes, scales, zeros, s); break;
+    case 512: quantize_int4_typed<T, 16>(W, N, K, sym, codes, scales, zeros, s); break;
+    case 1024: quantize_int4_typed<T, 32>(W, N, K, sym, codes, scales, zeros, s); break;
+    default: return WQ_ERR_UNSUPPORTED;
+  }
+  WQ_LAUNCH_CHECK("quantize_int4_kernel");
+  return WQ_OK;
+}
+
+int launch_quantize_int4(const void* W, int w_dtype, int64_t N, int64_t K, int gs, int sym,
+                         void* codes, void* scales, void* zeros, cudaStream_t s) {
+  switch (w_dtype) {
+    case WQ_F32: return quantize_int4_dispatch<float>(W, N, K, gs, sym, codes, scales, zeros, s);
+    case WQ_BF16:
+      return quantize_int4_dispatch<__nv_bfloat16>(W, N, K, gs, sym, codes, scales, zeros, s);
+    case WQ_F16: return quantize_int4_dispatch<__half>(W, N, K, gs, sym, codes, scales, zeros, s);
+  }
+  return WQ_ERR_ARG;
+}
+
+int launch_quantize_rows_i8(const void* W, int w_dtype, int64_t N, int64_t K, bool activation,
+                            void* q, void* scales, cudaStream_t s) {
+  const int grid = int(N < int64_t(sm_count()) * 16 ? N : int64_t(sm_count()) * 16);
+  int* st = status_ptr();
+  auto* qo = static_cast<int8_t*>(q);
+  auto* so = static_cast<float*>(scales);
+#define WQ_ROWS(T)                                                                           \
+  do {                                                                                       \
+    if (activation)                                                                          \
+      wq::quantize_rows_i8_kernel<T, true><<<grid, 256, 0, s>>>(static_cast<const T*>(W), N, \
+                                                                K, qo, so, st);              \
+    else                                                                                     \
+      wq::quantize_rows_i8_kernel<T, false><<<grid, 256, 0, s>>>(static_cast<const T*>(W),   \
+                                                                 N, K, qo, so, st);          \
+  } while (0)
+  switch (w_dtype) {
+    case WQ_F32: WQ_ROWS(float); break;
+    case WQ_BF16: WQ_ROWS(__nv_bfloat16); break;
+    case WQ_F16: WQ_ROWS(__half); break;
+    default: return WQ_ERR_ARG;
+  }
+#undef WQ_ROWS
+  WQ_LAUNCH_CHECK("quantize_rows_i8_kernel");
+  return WQ_OK;
+}
+
+int launch_dequant_int4(const void* codes, const void* scales, const void* zeros, int64_t N,
+                        int64_t K, int gs, int sym, void* out, int out_dtype, cudaStream_t s) {
+  const int grid = grid_for(N * (K / 32), 256);
+  auto* c = static_cast<const uint8_t*>(codes);
+  auto* sc = static_cast<const __half*>(scales);
+  auto* z = static_cast<const __half*>(zeros);
+  if (out_dtype == WQ_F32)
+    wq::dequant_int4_kernel<float><<<grid, 256, 0, s>>>(c, sc, z, N, K, gs, sym,
+                                                        static_cast<float*>(out));
+  else
+    wq::dequant_int4_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        c, sc, z, N, K, gs, sym, static_cast<__nv_bfloat16*>(out));
+  WQ_LAUNCH_CHECK("dequant_int4_kernel");
+  return WQ_OK;
+}
+
+int launch_dequant_int8_rows(const void* q, const void* scales, int64_t N, int64_t K, void* out,
+                             int out_dtype, cudaStream_t s) {
+  const int grid = grid_for(N * (K / 16), 256);
+  auto* qi = static_cast<const int8_t*>(q);
+  auto* sc = static_cast<const float*>(scales);
+  if (out_dtype == WQ_F32)
+    wq::dequant_int8_rows_kernel<float><<<grid, 256, 0, s>>>(qi, sc, N, K,
+                                                             static_cast<float*>(out));
+  else
+    wq::dequant_int8_rows_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        qi, sc, N, K, static_cast<__nv_bfloat16*>(out));
+  WQ_LAUNCH_CHECK("dequant_int8_rows_kernel");
+  return WQ_OK;
+}
+
+}  // namespace wq_host

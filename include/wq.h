@@ -1,0 +1,167 @@
+/*
+ * wq.h -- C ABI of libwq: group-wise affine weight quantization and the
+ * fused-dequantize W4A16 / W8A8 matrix products on NVIDIA B200 (sm_100a).
+ *
+ * Page tags used in the citations below (quantization write-ups this library
+ * implements):
+ *   [P1] "大模型量化技术入门：为什么我们需要量化？"
+ *   [P2] "从0到1：大模型量化"
+ *   [P3] "从 FP32 到 INT4：大模型推理加速中的量化优化实战路径"
+ *   [P4] "27届大模型面试准备（十九）：模型量化全攻略"
+ *   [P5] "大模型量化技术定义与主流方案解析"
+ *
+ * Conventions for every entry point:
+ *   - All tensor arguments are DEVICE pointers to row-major buffers that the
+ *     caller allocates and owns.  The library keeps no pointer after return.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously on that stream.
+ *   - The return value reports host-side argument validation and launch
+ *     errors (wq_status).  Errors the kernels detect (non-finite input, a
+ *     scale that overflows fp16, a bounded wait that gave up) are recorded in
+ *     a library-owned device status word read by wq_get_device_status().
+ *   - Pointers must be 16-byte aligned (WQ_ERR_ALIGN otherwise).
+ *   - Sizes are int64_t; negative sizes are WQ_ERR_ARG.  Empty problems
+ *     (N == 0 or M == 0) return WQ_OK and launch nothing.
+ *   - There is no CPU fallback: the calls need an sm_100a device.
+ *
+ * INT4 storage (the pages leave it open; this library fixes it):
+ *   codes  : uint8 [N, K/2]; element k of row n is the nibble in byte
+ *            n*K/2 + k/2, low nibble = even k; the nibble is the unsigned code
+ *            u = q - qmin (symmetric: u = q + 8, q in [-8, 7]; asymmetric:
+ *            u = q, q in [0, 15]).
+ *   scales : fp16 [N, K/group_size], one per group of group_size consecutive
+ *            input columns of a row.
+ *   zeros  : fp16 [N, K/group_size] integer-valued zero points in [0, 15]
+ *            (asymmetric only; NULL for symmetric).
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define WQ_API __attribute__((visibility("default")))
+#else
+#define WQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WQ_OK = 0,
+  WQ_ERR_ARG = -1,         /* bad size, NULL pointer, inconsistent options */
+  WQ_ERR_UNSUPPORTED = -2, /* valid in principle, not implemented (e.g. g != 128 in a GEMM) */
+  WQ_ERR_ALIGN = -3,       /* pointer not 16-byte aligned, or K not a multiple the kernel needs */
+  WQ_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed */
+  WQ_ERR_NONFINITE = -5,   /* device: NaN/Inf input, or a scale that overflows fp16 */
+  WQ_ERR_TIMEOUT = -6,     /* device: a bounded wait inside a kernel gave up */
+  WQ_ERR_WORKSPACE = -8,   /* workspace pointer NULL or too small */
+  WQ_ERR_NO_DEVICE = -9    /* the current device is not sm_100 */
+} wq_status;
+
+typedef enum { WQ_F32 = 0, WQ_BF16 = 1, WQ_F16 = 2 } wq_dtype;
+
+/*
+ * wq_quantize_pack -- quantize a weight matrix W [N, K].
+ *
+ * bits == 4: group-wise affine INT4 ([P4] sec. 2.1 affine quantization,
+ *   sec. 2.2 per-group g=128; [P3] sec. 2.1 symmetric/asymmetric quantizers,
+ *   sec. 2.2 per-group granularity).  For each row n and group j of
+ *   group_size columns:
+ *     sym : s = fp16(amax / 7); q = clamp(round(x / s), -8, 7)
+ *     asym: s = fp16((max - min) / 15); z = clamp(round(-min / s), 0, 15);
+ *           q = clamp(round(x / s) + z, 0, 15)
+ *   round = half to even; x / s is one IEEE fp32 division by the stored fp16
+ *   scale.  Degenerate groups ([P3] sec. 2.1): sym with amax < 1e-8 (or an
+ *   fp16 scale of zero) -> q = 0, stored scale fp16(amax); asym with
+ *   max - min < 1e-8 (or an fp16 scale of zero) -> q = 0, s = 1, z = 0.
+ *   Outputs: codes uint8 [N, K/2], scales fp16 [N, K/g], zeros fp16 [N, K/g]
+ *   (asym) -- zeros must be NULL iff sym.
+ *   Requires K % group_size == 0, group_size % 32 == 0.
+ * bits == 8: symmetric INT8 with one fp32 scale per output row ([P4] sec. 2.2,
+ *   per-channel weights): s = amax / 127, q = clamp(round(x / s), -127, 127);
+ *   rows with amax < 1e-8 get q = 0 and s = amax.  Requires sym == 1,
+ *   group_size == K, zeros == NULL.  Outputs: codes int8 [N, K], scales fp32 [N].
+ *
+ * W: w_dtype WQ_F32, WQ_BF16 or WQ_F16, row-major [N, K].
+ * Errors: WQ_ERR_ARG (sizes, NULL, sym/zeros mismatch), WQ_ERR_UNSUPPORTED
+ * (bits not 4/8), WQ_ERR_ALIGN; device: WQ_ERR_NONFINITE (codes of the
+ * offending group are then unspecified).
+ */
+WQ_API int wq_quantize_pack(const void *W, int w_dtype, int64_t N, int64_t K,
+                     int group_size, int bits, int sym, void *codes,
+                     void *scales, void *zeros, void *stream);
+
+/*
+ * wq_dequant -- x_hat = s * (q - z) ([P2] sec. 2 dequantization; [P4]
+ * sec. 2.1).  bits == 4: inputs as produced by wq_quantize_pack (zeros NULL
+ * iff sym); the fp32 result is exact.  bits == 8: x_hat = s[n] * q (int8
+ * codes, fp32 scales, group_size == K, sym == 1).
+ * out: [N, K] of out_dtype WQ_F32 or WQ_BF16 (the fp32 value rounded to
+ * nearest even).
+ */
+WQ_API int wq_dequant(const void *codes, const void *scales, const void *zeros,
+               int64_t N, int64_t K, int group_size, int bits, int sym,
+               void *out, int out_dtype, void *stream);
+
+/*
+ * wq_gemm_w4a16 -- Y = X * dequant(W)^T with INT4 group-wise weights and
+ * bf16 activations ([P4] sec. 2.3 W4A16; [P5] sec. 四 fused dequantization:
+ * the weight is expanded tile by tile inside the kernel and never written back
+ * to memory).  X bf16 [M, K]; codes/scales/zeros as above with
+ * group_size == 128 (others: WQ_ERR_UNSUPPORTED, [P4] sec. 7.2: the group must
+ * divide the kernel tile); Y bf16 [M, N]; fp32 accumulation.
+ * M <= 16 runs the decode kernel (weights streamed once from HBM); larger M
+ * runs the tensor-core GEMM.  Requires K % 128 == 0 and N % 8 == 0.
+ */
+WQ_API int wq_gemm_w4a16(const void *X, int64_t M, int64_t K, const void *codes,
+                  const void *scales, const void *zeros, int64_t N,
+                  int group_size, int sym, void *Y, void *stream);
+
+/*
+ * wq_quant_act_i8 -- per-token dynamic INT8 quantization of activations
+ * ([P4] sec. 6 per-token absmax quantizer, used for the A8 of W8A8, [P4]
+ * sec. 2.3): s[m] = max(amax_m / 127, 1e-8); q = clamp(round(x / s), -128, 127).
+ * X bf16 [M, K] -> q int8 [M, K], s fp32 [M].  Requires K % 16 == 0.
+ */
+WQ_API int wq_quant_act_i8(const void *X, int64_t M, int64_t K, void *q, void *s,
+                    void *stream);
+
+/* Bytes of workspace wq_gemm_w8a8 needs: int8 X [M, K] then fp32 scales [M],
+ * each part 256-byte aligned. */
+WQ_API size_t wq_w8a8_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * wq_gemm_w8a8 -- W8A8 product on the int8 tensor cores ([P4] sec. 2.3 and
+ * 4.2: int8 weights and activations, int32 accumulation, then a floating
+ * rescale).  X bf16 [M, K] is quantized per token into `ws` (see
+ * wq_quant_act_i8), then acc[m, n] = sum_k qx[m, k] * qw[n, k] (int32) and
+ * Y[m, n] = bf16(float(acc) * sx[m] * w_scales[n]).
+ * Wq int8 [N, K] and w_scales fp32 [N] come from wq_quantize_pack(bits = 8).
+ * acc_out (nullable) receives the raw int32 accumulators [M, N].
+ * Requires K % 128 == 0, N % 16 == 0, ws of wq_w8a8_workspace_bytes(M, K).
+ */
+WQ_API int wq_gemm_w8a8(const void *X, int64_t M, int64_t K, const void *Wq,
+                 const void *w_scales, int64_t N, void *Y, void *ws,
+                 size_t ws_bytes, void *acc_out, void *stream);
+
+/*
+ * wq_get_device_status -- synchronize `stream`, then return the first error
+ * any kernel recorded since the last reset (WQ_OK if none); clear it when
+ * reset != 0.  Returns WQ_ERR_CUDA if the synchronization itself fails.
+ */
+WQ_API int wq_get_device_status(void *stream, int reset);
+
+/* Human-readable name of a wq_status value (static storage). */
+WQ_API const char *wq_status_str(int status);
+
+/* Text of the last CUDA error seen on the host side by this thread. */
+WQ_API const char *wq_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WQ_H */

@@ -1,0 +1,99 @@
+"""The C-ABI library loads, exports every symbol include/wq.h declares, and
+rejects bad arguments on the host (no GPU needed: validation returns before
+any CUDA call; no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_gemm_group_b200 as wq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    wq.build()
+    return wq.lib()
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "wq.h")).read()
+    return sorted(set(re.findall(r"WQ_API\s+[\w\s\*]*?\b(wq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_python_list():
+    assert _declared_symbols() == sorted(wq.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in _declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code, name in [(0, "WQ_OK"), (-1, "WQ_ERR_ARG"), (-2, "WQ_ERR_UNSUPPORTED"),
+                       (-3, "WQ_ERR_ALIGN"), (-6, "WQ_ERR_TIMEOUT"), (-9, "WQ_ERR_NO_DEVICE")]:
+        assert wq.wq_status_str(code) == name
+
+
+def test_workspace_size(L):
+    assert wq.wq_w8a8_workspace_bytes(4096, 4096) == 4096 * 4096 + 4096 * 4
+    assert wq.wq_w8a8_workspace_bytes(3, 128) == 512 + 256
+    assert wq.wq_w8a8_workspace_bytes(0, 128) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def test_quantize_validation(L):
+    q = L.wq_quantize_pack
+    assert q(FAKE, 1, -1, 128, 128, 4, 1, FAKE, FAKE, None, None) == wq.WQ_ERR_ARG
+    assert q(FAKE, 1, 8, 200, 128, 4, 1, FAKE, FAKE, None, None) == wq.WQ_ERR_ARG      # K % g
+    assert q(FAKE, 1, 8, 256, 128, 4, 1, FAKE, FAKE, FAKE, None) == wq.WQ_ERR_ARG      # sym with zeros
+    assert q(FAKE, 1, 8, 256, 128, 4, 0, FAKE, FAKE, None, None) == wq.WQ_ERR_ARG      # asym w/o zeros
+    assert q(FAKE, 1, 8, 240, 48, 4, 1, FAKE, FAKE, None, None) == wq.WQ_ERR_UNSUPPORTED
+    assert q(FAKE, 1, 8, 256, 128, 3, 1, FAKE, FAKE, None, None) == wq.WQ_ERR_UNSUPPORTED
+    assert q(FAKE, 7, 8, 256, 128, 4, 1, FAKE, FAKE, None, None) == wq.WQ_ERR_ARG      # dtype
+    assert q(MISALIGNED, 1, 8, 256, 128, 4, 1, FAKE, FAKE, None, None) == wq.WQ_ERR_ALIGN
+    assert q(FAKE, 1, 8, 256, 256, 8, 0, FAKE, FAKE, None, None) == wq.WQ_ERR_ARG      # int8 asym
+    assert q(FAKE, 1, 8, 256, 128, 8, 1, FAKE, FAKE, None, None) == wq.WQ_ERR_ARG      # int8 g != K
+    assert q(None, 1, 0, 256, 128, 4, 1, None, None, None, None) == wq.WQ_OK          # empty
+
+
+def test_dequant_validation(L):
+    d = L.wq_dequant
+    assert d(FAKE, FAKE, None, 8, 256, 128, 4, 1, FAKE, 2, None) == wq.WQ_ERR_ARG       # fp16 out
+    assert d(FAKE, FAKE, FAKE, 8, 256, 128, 4, 1, FAKE, 0, None) == wq.WQ_ERR_ARG
+    assert d(FAKE, FAKE, None, 0, 256, 128, 4, 1, FAKE, 0, None) == wq.WQ_OK
+
+
+def test_gemm_w4a16_validation(L):
+    g = L.wq_gemm_w4a16
+    assert g(FAKE, 1, 4096, FAKE, FAKE, None, 4096, 64, 1, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
+    assert g(FAKE, 1, 4000, FAKE, FAKE, None, 4096, 128, 1, FAKE, None) == wq.WQ_ERR_ALIGN
+    assert g(FAKE, 1, 4096, FAKE, FAKE, None, 4100, 128, 1, FAKE, None) == wq.WQ_ERR_ALIGN
+    assert g(FAKE, 1, 4096, FAKE, FAKE, FAKE, 4096, 128, 1, FAKE, None) == wq.WQ_ERR_ARG
+    assert g(FAKE, 0, 4096, FAKE, FAKE, None, 4096, 128, 1, FAKE, None) == wq.WQ_OK
+    assert g(MISALIGNED, 1, 4096, FAKE, FAKE, None, 4096, 128, 1, FAKE, None) == wq.WQ_ERR_ALIGN
+
+
+def test_act_quant_validation(L):
+    a = L.wq_quant_act_i8
+    assert a(FAKE, 4, 100, FAKE, FAKE, None) == wq.WQ_ERR_ALIGN
+    assert a(FAKE, -4, 128, FAKE, FAKE, None) == wq.WQ_ERR_ARG
+    assert a(FAKE, 0, 128, FAKE, FAKE, None) == wq.WQ_OK
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    W = torch.zeros(8, 256)
+    with pytest.raises(wq.WQError):
+        wq.quantize_pack(W)
+
+
+def test_oracle_builds():
+    import oracle
+    assert os.path.exists(oracle.build.build())

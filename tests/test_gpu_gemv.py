@@ -1,0 +1,86 @@
+"""GPU parity of the W4A16 decode product (M <= 16) against the fp64 oracle:
+max_{m,n} |Y - Y_ref| / ||Y_ref[m, :]||_2 <= 2e-3, on the workloads' full
+shapes (sampled output columns for the 70B shapes) and on ragged cases."""
+import numpy as np
+import pytest
+import torch
+
+import bit_gemm_group_b200 as wq
+import oracle
+from parity_util import REL_ROW_TOL, oracle_input, rel_row_error
+from workloads import WORKLOADS, make_activation, make_weight, bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    wq.wq_get_device_status(reset=True)
+    yield
+    assert wq.wq_get_device_status(reset=True) == wq.WQ_OK
+
+
+def quantized(W, sym):
+    codes, scales, zeros = wq.quantize_pack(W.cuda(), 128, 4, sym)
+    arr, tag = oracle_input(W)
+    oc, osc, oz, _ = oracle.quantize_int4(arr, 128, sym, dtype_tag=tag)
+    return (codes, scales, zeros), (oc, osc, oz)
+
+
+def check_gemv(X, dev_q, ora_q, sym, windows=None):
+    codes, scales, zeros = dev_q
+    Y = wq.gemm_w4a16(X.cuda(), codes, scales, zeros, 128, sym).float().cpu().numpy()
+    N = codes.shape[0]
+    windows = windows or [(0, N)]
+    for n0, n1 in windows:
+        Yref, st = oracle.gemm_w4a16(bf16_bits(X), *ora_q, 128, sym, n0, n1)
+        assert st == oracle.OK
+        err = rel_row_error(Y[:, n0:n1], Yref)
+        assert err <= REL_ROW_TOL, (n0, n1, err)
+    return Y
+
+
+def test_tiny_workload():
+    wl = WORKLOADS["tiny"]
+    W = wl.weight(0)
+    dq, oq = quantized(W, wl.sym)
+    check_gemv(wl.activation(1, 512), dq, oq, wl.sym)
+
+
+@pytest.mark.parametrize("i", [0, 1, 2])
+def test_7b_decode_full(i):
+    wl = WORKLOADS["7b-decode"]
+    W = wl.weight(i)
+    dq, oq = quantized(W, True)
+    for M in wl.ms:
+        check_gemv(wl.activation(M, W.shape[1]), dq, oq, True)
+
+
+@pytest.mark.parametrize("i", [0, 1])
+def test_70b_decode_sampled(i):
+    wl = WORKLOADS["70b-decode"]
+    W = wl.weight(i)
+    N = W.shape[0]
+    dq, oq = quantized(W, False)
+    windows = [(0, 256), (N // 2 - 128, N // 2 + 128), (N - 256, N)]
+    for M in wl.ms:
+        check_gemv(wl.activation(M, W.shape[1]), dq, oq, False, windows)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 13, 16])
+@pytest.mark.parametrize("N,K", [(8, 128), (24, 256), (136, 1152), (264, 4096)])
+@pytest.mark.parametrize("sym", [True, False])
+def test_ragged(M, N, K, sym):
+    W = make_weight(N, K, 0.02, seed=N + K, outlier_frac=0.01, outlier_scale=30.0)
+    dq, oq = quantized(W, sym)
+    check_gemv(make_activation(M, K, seed=M), dq, oq, sym)
+
+
+def test_deterministic():
+    wl = WORKLOADS["7b-decode"]
+    W = wl.weight(1)
+    (codes, scales, zeros), _ = quantized(W, True)
+    X = wl.activation(4, W.shape[1]).cuda()
+    a = wq.gemm_w4a16(X, codes, scales, zeros)
+    b = wq.gemm_w4a16(X, codes, scales, zeros)
+    assert torch.equal(a, b)
