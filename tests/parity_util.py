@@ -26,8 +26,21 @@ def u16(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def rel_row_error(Y: np.ndarray, Yref: np.ndarray) -> float:
+def rel_row_error(Y: np.ndarray, Yref: np.ndarray, rounding_aware: bool = False) -> float:
+    """max_{m,n} |Y - Y_ref| / ||Y_ref[m, :]||_2.
+
+    With rounding_aware, each element's error is first reduced by half a bf16
+    ulp of Y_ref (the rounding of the bf16 output itself, up to 2^-8 of the
+    value): with very few outputs per row one element carries most of the row
+    norm and the output rounding alone can exceed the row-normalised bound.
+    The workloads' full-size checks use the plain bound."""
     Y = np.asarray(Y, np.float64)
+    err = np.abs(Y - Yref)
+    if rounding_aware:
+        mag = np.abs(Yref)
+        e = np.floor(np.log2(np.where(mag > 0, mag, 1.0)))
+        half_ulp = np.where(mag > 0, np.exp2(e - 8), 0.0)
+        err = np.maximum(err - half_ulp, 0.0)
     norms = np.linalg.norm(Yref, axis=1)
     norms = np.where(norms == 0, 1.0, norms)
-    return float((np.abs(Y - Yref).max(axis=1) / norms).max())
+    return float((err.max(axis=1) / norms).max())

@@ -27,7 +27,7 @@ def quantized(W, sym):
     return (codes, scales, zeros), (oc, osc, oz)
 
 
-def check_gemv(X, dev_q, ora_q, sym, windows=None):
+def check_gemv(X, dev_q, ora_q, sym, windows=None, rounding_aware=False):
     codes, scales, zeros = dev_q
     Y = wq.gemm_w4a16(X.cuda(), codes, scales, zeros, 128, sym).float().cpu().numpy()
     N = codes.shape[0]
@@ -35,7 +35,7 @@ def check_gemv(X, dev_q, ora_q, sym, windows=None):
     for n0, n1 in windows:
         Yref, st = oracle.gemm_w4a16(bf16_bits(X), *ora_q, 128, sym, n0, n1)
         assert st == oracle.OK
-        err = rel_row_error(Y[:, n0:n1], Yref)
+        err = rel_row_error(Y[:, n0:n1], Yref, rounding_aware)
         assert err <= REL_ROW_TOL, (n0, n1, err)
     return Y
 
@@ -73,7 +73,7 @@ def test_70b_decode_sampled(i):
 def test_ragged(M, N, K, sym):
     W = make_weight(N, K, 0.02, seed=N + K, outlier_frac=0.01, outlier_scale=30.0)
     dq, oq = quantized(W, sym)
-    check_gemv(make_activation(M, K, seed=M), dq, oq, sym)
+    check_gemv(make_activation(M, K, seed=M), dq, oq, sym, rounding_aware=N < 256)
 
 
 def test_deterministic():
