@@ -36,7 +36,7 @@ WQ_F32, WQ_BF16, WQ_F16 = 0, 1, 2
 EXPORTED = (
     "wq_quantize_pack", "wq_dequant", "wq_gemm_w4a16", "wq_quant_act_i8",
     "wq_w8a8_workspace_bytes", "wq_gemm_w8a8", "wq_get_device_status",
-    "wq_status_str", "wq_last_cuda_error",
+    "wq_status_str", "wq_last_cuda_error", "wq_selftest_wait_timeout",
 )
 
 
@@ -89,6 +89,8 @@ def _declare(L):
     L.wq_get_device_status.argtypes = [_P, _INT]
     L.wq_status_str.argtypes = [_INT]
     L.wq_status_str.restype = ctypes.c_char_p
+    L.wq_selftest_wait_timeout.argtypes = [_INT, _P]
+    L.wq_selftest_wait_timeout.restype = _INT
     L.wq_last_cuda_error.argtypes = []
     L.wq_last_cuda_error.restype = ctypes.c_char_p
     for name in ("wq_quantize_pack", "wq_dequant", "wq_gemm_w4a16", "wq_quant_act_i8",
@@ -173,6 +175,12 @@ def wq_gemm_w8a8(X, Wq, w_scales, Y, ws, acc_out=None, stream=None):
 def wq_get_device_status(reset=True, stream=None):
     """Synchronize the stream and return the first kernel-detected error code."""
     return int(lib().wq_get_device_status(_stream(stream), int(bool(reset))))
+
+
+def wq_selftest_wait_timeout(limit_us, stream=None):
+    """Launch the bounded-wait self-test kernel (records WQ_ERR_TIMEOUT)."""
+    _check(lib().wq_selftest_wait_timeout(int(limit_us), _stream(stream)),
+           "wq_selftest_wait_timeout")
 
 
 def wq_status_str(status):

@@ -74,6 +74,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Host-side helpers (defined in wq_api.cu)
 // ---------------------------------------------------------------------------
 namespace wq_host {
+// check (once per device) that the current device is sm_100 and set up the
+// status word; WQ_OK or an error status
+int ensure_device();
 // device pointer of the status word on the current device
 int* status_ptr();
 // number of SMs of the current device

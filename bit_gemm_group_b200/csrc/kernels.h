@@ -20,4 +20,7 @@ int launch_gemv_w4a16(const void* X, int64_t M, int64_t K, const void* codes,
                       const void* scales, const void* zeros, int64_t N, int sym, void* Y,
                       cudaStream_t s);
 
+int launch_gemm_w8a8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
+                     int64_t N, void* Y, void* ws, void* acc_out, cudaStream_t s);
+
 }  // namespace wq_host

@@ -191,9 +191,20 @@ size_t wq_w8a8_workspace_bytes(int64_t M, int64_t K) {
 
 int wq_gemm_w8a8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
                  int64_t N, void* Y, void* ws, size_t ws_bytes, void* acc_out, void* stream) {
-  (void)X; (void)M; (void)K; (void)Wq; (void)w_scales; (void)N; (void)Y; (void)ws;
-  (void)ws_bytes; (void)acc_out; (void)stream;
-  return WQ_ERR_UNSUPPORTED;
+  if (M < 0 || K < 0 || N < 0) return WQ_ERR_ARG;
+  if ((K % 16) != 0 || (N % 16) != 0) return WQ_ERR_ALIGN;
+  if (M > (int64_t(1) << 31) / 2 || N > (int64_t(1) << 31) / 2 || K > (int64_t(1) << 24))
+    return WQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return WQ_OK;
+  if (K == 0) return WQ_ERR_ARG;
+  if (!X || !Wq || !w_scales || !Y) return WQ_ERR_ARG;
+  if (!ws || ws_bytes < wq_w8a8_workspace_bytes(M, K)) return WQ_ERR_WORKSPACE;
+  if (!aligned16(X) || !aligned16(Wq) || !aligned16(w_scales) || !aligned16(Y) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || (acc_out && !aligned16(acc_out)))
+    return WQ_ERR_ALIGN;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  return wq_host::launch_gemm_w8a8(X, M, K, Wq, w_scales, N, Y, ws, acc_out, as_stream(stream));
 }
 
 int wq_get_device_status(void* stream, int reset) {

@@ -155,6 +155,17 @@ WQ_API int wq_gemm_w8a8(const void *X, int64_t M, int64_t K, const void *Wq,
  */
 WQ_API int wq_get_device_status(void *stream, int reset);
 
+/*
+ * wq_selftest_wait_timeout -- exercises the bounded-wait path that every
+ * tensor-core kernel of this library uses for its pipeline barriers.  It
+ * launches one CTA that waits on a barrier nothing will ever complete; after
+ * limit_us microseconds (1 .. 1e6) the wait gives up, records WQ_ERR_TIMEOUT in
+ * the device status word and the kernel returns normally (no fault, the
+ * context stays usable).  Read the result with wq_get_device_status().
+ * The quantization pages have no counterpart: this is a failure-detection hook.
+ */
+WQ_API int wq_selftest_wait_timeout(int limit_us, void *stream);
+
 /* Human-readable name of a wq_status value (static storage). */
 WQ_API const char *wq_status_str(int status);
 
