@@ -133,7 +133,8 @@ def setup_decode(wq, wl, M, dev, rot):
                            None if zeros is None else zeros.clone()))
         X = wl.activation(M, K).to(dev)
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        sets.append({"N": N, "K": K, "copies": copies, "X": X, "Y": Y})
+        ws = wq.w4a16_workspace(M, N, K, dev)
+        sets.append({"N": N, "K": K, "copies": copies, "X": X, "Y": Y, "ws": ws})
     return sets
 
 
@@ -147,7 +148,7 @@ def capture_shape_graph(wq, s, sym, count, start):
         with torch.cuda.graph(g, stream=stream):
             for j in range(count):
                 c, sc, z = s["copies"][(start + j) % len(s["copies"])]
-                wq.wq_gemm_w4a16(s["X"], c, sc, z, s["N"], 128, sym, s["Y"])
+                wq.wq_gemm_w4a16(s["X"], c, sc, z, s["N"], 128, sym, s["Y"], s["ws"])
     torch.cuda.current_stream().wait_stream(stream)
     return g
 
@@ -199,7 +200,7 @@ def run_ours(args, rank, world, local_rank):
         for r in range(rem):
             for s in sets:
                 c, sc, z = s["copies"][r % ROT]
-                wq.wq_gemm_w4a16(s["X"], c, sc, z, s["N"], 128, wl.sym, s["Y"])
+                wq.wq_gemm_w4a16(s["X"], c, sc, z, s["N"], 128, wl.sym, s["Y"], s["ws"])
 
     warm = max(3, args.warmup)
     run_steps(warm)
@@ -287,7 +288,7 @@ def measure_e2e(wq, sets, wl, M, dev, steps=200):
         for j, s in enumerate(sets):
             s["X"].copy_(host_x[j], non_blocking=True)
             c, sc, z = s["copies"][i % len(s["copies"])]
-            wq.wq_gemm_w4a16(s["X"], c, sc, z, s["N"], 128, wl.sym, s["Y"])
+            wq.wq_gemm_w4a16(s["X"], c, sc, z, s["N"], 128, wl.sym, s["Y"], s["ws"])
             host_y[j].copy_(s["Y"], non_blocking=True)
 
     for i in range(5):

@@ -34,7 +34,8 @@ WQ_F32, WQ_BF16, WQ_F16 = 0, 1, 2
 
 # every symbol include/wq.h declares
 EXPORTED = (
-    "wq_quantize_pack", "wq_dequant", "wq_gemm_w4a16", "wq_quant_act_i8",
+    "wq_quantize_pack", "wq_dequant", "wq_w4a16_workspace_bytes", "wq_gemm_w4a16",
+    "wq_quant_act_i8",
     "wq_w8a8_workspace_bytes", "wq_gemm_w8a8", "wq_get_device_status",
     "wq_status_str", "wq_last_cuda_error", "wq_selftest_wait_timeout",
 )
@@ -81,7 +82,9 @@ _SZ = ctypes.c_size_t
 def _declare(L):
     L.wq_quantize_pack.argtypes = [_P, _INT, _I64, _I64, _INT, _INT, _INT, _P, _P, _P, _P]
     L.wq_dequant.argtypes = [_P, _P, _P, _I64, _I64, _INT, _INT, _INT, _P, _INT, _P]
-    L.wq_gemm_w4a16.argtypes = [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _INT, _P, _P]
+    L.wq_w4a16_workspace_bytes.argtypes = [_I64, _I64, _I64]
+    L.wq_w4a16_workspace_bytes.restype = _SZ
+    L.wq_gemm_w4a16.argtypes = [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _INT, _P, _P, _SZ, _P]
     L.wq_quant_act_i8.argtypes = [_P, _I64, _I64, _P, _P, _P]
     L.wq_w8a8_workspace_bytes.argtypes = [_I64, _I64]
     L.wq_w8a8_workspace_bytes.restype = _SZ
@@ -147,10 +150,16 @@ def wq_dequant(codes, scales, zeros, N, K, group_size, bits, sym, out, stream=No
     _check(st, "wq_dequant")
 
 
-def wq_gemm_w4a16(X, codes, scales, zeros, N, group_size, sym, Y, stream=None):
+def wq_w4a16_workspace_bytes(M, N, K):
+    return int(lib().wq_w4a16_workspace_bytes(M, N, K))
+
+
+def wq_gemm_w4a16(X, codes, scales, zeros, N, group_size, sym, Y, ws=None, stream=None):
     M, K = X.shape
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     st = lib().wq_gemm_w4a16(_ptr(X), M, K, _ptr(codes), _ptr(scales), _ptr(zeros), N,
-                             group_size, int(bool(sym)), _ptr(Y), _stream(stream))
+                             group_size, int(bool(sym)), _ptr(Y), _ptr(ws), ws_bytes,
+                             _stream(stream))
     _check(st, "wq_gemm_w4a16")
 
 
@@ -219,11 +228,19 @@ def dequant(codes, scales, zeros, K, group_size=128, bits=4, sym=True,
     return out
 
 
-def gemm_w4a16(X, codes, scales, zeros, group_size=128, sym=True):
-    M = X.shape[0]
+def w4a16_workspace(M, N, K, device):
+    """A zero-filled workspace for wq_gemm_w4a16 (None when M > 16)."""
+    n = wq_w4a16_workspace_bytes(M, N, K)
+    return torch.zeros((n,), dtype=torch.uint8, device=device) if n else None
+
+
+def gemm_w4a16(X, codes, scales, zeros, group_size=128, sym=True, ws=None):
+    M, K = X.shape
     N = codes.shape[0]
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
-    wq_gemm_w4a16(X, codes, scales, zeros, N, group_size, sym, Y)
+    if ws is None:
+        ws = w4a16_workspace(M, N, K, X.device)
+    wq_gemm_w4a16(X, codes, scales, zeros, N, group_size, sym, Y, ws)
     return Y
 
 

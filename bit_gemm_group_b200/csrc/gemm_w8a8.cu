@@ -209,10 +209,10 @@ int launch_gemm_w8a8(const void* X, int64_t M, int64_t K, const void* Wq, const 
 
   CUtensorMap ta, tb;
   st = make_tmap_2d(&ta, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(M), uint64_t(K), BM, BK,
-                    true);
+                    128);
   if (st != WQ_OK) return st;
   st = make_tmap_2d(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(N), uint64_t(K), BN, BK,
-                    true);
+                    128);
   if (st != WQ_OK) return st;
 
   static bool attr_done[64] = {};

@@ -302,11 +302,11 @@ __host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
 namespace wq_host {
 
 // 2D row-major tensor [rows, cols] of `elem_bytes`-byte elements; the box is
-// [box_rows, box_cols]; 128-byte swizzle unless `swizzle128` is false.
+// [box_rows, box_cols]; swizzle_bytes is 0 (none), 64 or 128.
 // Returns WQ_OK or WQ_ERR_CUDA.
 int make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
                  uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
-                 bool swizzle128);
+                 int swizzle_bytes);
 
 // Time budget of one kernel launch for its bounded waits, in ns (2 s; the
 // environment variable WQ_WAIT_LIMIT_MS overrides it).

@@ -1,6 +1,7 @@
 // wq_api.cu -- the C ABI declared in include/wq.h: argument validation,
 // dispatch to the kernels, and the device status word.
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -150,24 +151,34 @@ int wq_dequant(const void* codes, const void* scales, const void* zeros, int64_t
                                            as_stream(stream));
 }
 
+size_t wq_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || M > 16 || N <= 0 || K < 128) return 0;
+  if (wq_host::ensure_device() != WQ_OK) return 0;
+  return wq_host::gemv_workspace_bytes(N, K);
+}
+
 int wq_gemm_w4a16(const void* X, int64_t M, int64_t K, const void* codes, const void* scales,
-                  const void* zeros, int64_t N, int group_size, int sym, void* Y, void* stream) {
+                  const void* zeros, int64_t N, int group_size, int sym, void* Y, void* ws,
+                  size_t ws_bytes, void* stream) {
   if (M < 0 || K < 0 || N < 0) return WQ_ERR_ARG;
   if (sym != 0 && sym != 1) return WQ_ERR_ARG;
   if ((sym == 1) != (zeros == nullptr)) return WQ_ERR_ARG;
   if (group_size != 128) return WQ_ERR_UNSUPPORTED;
   if ((K % 128) != 0 || (N % 8) != 0) return WQ_ERR_ALIGN;
+  if (N > (int64_t(1) << 30) || K > (int64_t(1) << 24)) return WQ_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return WQ_OK;
   if (K == 0) return WQ_ERR_ARG;
   if (!X || !codes || !scales || !Y) return WQ_ERR_ARG;
   if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(Y) ||
-      (zeros && !aligned16(zeros)))
+      (zeros && !aligned16(zeros)) || (ws && (reinterpret_cast<uintptr_t>(ws) & 255u)))
     return WQ_ERR_ALIGN;
   int st = wq_host::ensure_device();
   if (st != WQ_OK) return st;
-  if (M <= 16)
-    return wq_host::launch_gemv_w4a16(X, M, K, codes, scales, zeros, N, sym, Y,
-                                      as_stream(stream));
+  if (M <= 16) {
+    if (!ws || ws_bytes < wq_host::gemv_workspace_bytes(N, K)) return WQ_ERR_WORKSPACE;
+    return wq_host::launch_gemv_w4a16_tc(X, M, K, codes, scales, zeros, N, sym, Y, ws,
+                                         as_stream(stream));
+  }
   return WQ_ERR_UNSUPPORTED;
 }
 

@@ -114,12 +114,22 @@ WQ_API int wq_dequant(const void *codes, const void *scales, const void *zeros,
  * to memory).  X bf16 [M, K]; codes/scales/zeros as above with
  * group_size == 128 (others: WQ_ERR_UNSUPPORTED, [P4] sec. 7.2: the group must
  * divide the kernel tile); Y bf16 [M, N]; fp32 accumulation.
- * M <= 16 runs the decode kernel (weights streamed once from HBM); larger M
- * runs the tensor-core GEMM.  Requires K % 128 == 0 and N % 8 == 0.
+ * M <= 16 runs the decode kernel (every weight byte streamed once from HBM,
+ * the work split evenly over all SMs); larger M runs the tensor-core GEMM.
+ * Requires K % 128 == 0 and N % 8 == 0.
+ *
+ * ws / ws_bytes: device workspace of wq_w4a16_workspace_bytes(M, N, K) bytes
+ * (0 for M > 16, where ws may be NULL).  Fill it with zeros once before its
+ * first use (e.g. cudaMemset); every call that completes leaves it zeroed
+ * again, so it can be reused call after call.  Calls that may run at the same
+ * time on the GPU need separate workspaces.  After a call reported
+ * WQ_ERR_TIMEOUT, zero it again.  WQ_ERR_WORKSPACE if NULL or too small.
  */
+WQ_API size_t wq_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 WQ_API int wq_gemm_w4a16(const void *X, int64_t M, int64_t K, const void *codes,
-                  const void *scales, const void *zeros, int64_t N,
-                  int group_size, int sym, void *Y, void *stream);
+                         const void *scales, const void *zeros, int64_t N,
+                         int group_size, int sym, void *Y, void *ws,
+                         size_t ws_bytes, void *stream);
 
 /*
  * wq_quant_act_i8 -- per-token dynamic INT8 quantization of activations

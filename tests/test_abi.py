@@ -72,12 +72,13 @@ def test_dequant_validation(L):
 
 def test_gemm_w4a16_validation(L):
     g = L.wq_gemm_w4a16
-    assert g(FAKE, 1, 4096, FAKE, FAKE, None, 4096, 64, 1, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
-    assert g(FAKE, 1, 4000, FAKE, FAKE, None, 4096, 128, 1, FAKE, None) == wq.WQ_ERR_ALIGN
-    assert g(FAKE, 1, 4096, FAKE, FAKE, None, 4100, 128, 1, FAKE, None) == wq.WQ_ERR_ALIGN
-    assert g(FAKE, 1, 4096, FAKE, FAKE, FAKE, 4096, 128, 1, FAKE, None) == wq.WQ_ERR_ARG
-    assert g(FAKE, 0, 4096, FAKE, FAKE, None, 4096, 128, 1, FAKE, None) == wq.WQ_OK
-    assert g(MISALIGNED, 1, 4096, FAKE, FAKE, None, 4096, 128, 1, FAKE, None) == wq.WQ_ERR_ALIGN
+    assert g(FAKE, 1, 4096, FAKE, FAKE, None, 4096, 64, 1, FAKE, FAKE, 1 << 20, None) == wq.WQ_ERR_UNSUPPORTED
+    assert g(FAKE, 1, 4000, FAKE, FAKE, None, 4096, 128, 1, FAKE, FAKE, 1 << 20, None) == wq.WQ_ERR_ALIGN
+    assert g(FAKE, 1, 4096, FAKE, FAKE, None, 4100, 128, 1, FAKE, FAKE, 1 << 20, None) == wq.WQ_ERR_ALIGN
+    assert g(FAKE, 1, 4096, FAKE, FAKE, FAKE, 4096, 128, 1, FAKE, FAKE, 1 << 20, None) == wq.WQ_ERR_ARG
+    assert g(FAKE, 0, 4096, FAKE, FAKE, None, 4096, 128, 1, FAKE, None, 0, None) == wq.WQ_OK
+    assert g(MISALIGNED, 1, 4096, FAKE, FAKE, None, 4096, 128, 1, FAKE, FAKE, 1 << 20, None) == wq.WQ_ERR_ALIGN
+    assert g(FAKE, 1, 4096, FAKE, FAKE, None, 4096, 128, 1, FAKE, MISALIGNED, 1 << 20, None) == wq.WQ_ERR_ALIGN
 
 
 def test_act_quant_validation(L):

@@ -76,6 +76,28 @@ def test_ragged(M, N, K, sym):
     check_gemv(make_activation(M, K, seed=M), dq, oq, sym, rounding_aware=N < 256)
 
 
+def test_workspace_reused_and_left_zeroed():
+    W = make_weight(1000 * 8, 4096, 0.02, seed=3)
+    dq, oq = quantized(W, True)
+    codes, scales, zeros = dq
+    X = make_activation(2, 4096, seed=4).cuda()
+    ws = wq.w4a16_workspace(2, W.shape[0], 4096, "cuda")
+    outs = [wq.gemm_w4a16(X, codes, scales, zeros, ws=ws) for _ in range(3)]
+    assert all(torch.equal(outs[0], o) for o in outs[1:])
+    T = (W.shape[0] + 127) // 128
+    assert int(ws[: 4 * T].count_nonzero()) == 0  # arrival counters reset by every call
+
+
+def test_workspace_too_small():
+    W = make_weight(256, 1024, 0.02, seed=3).cuda()
+    codes, scales, _ = wq.quantize_pack(W, 128, 4, True)
+    X = make_activation(1, 1024, seed=4).cuda()
+    Y = torch.empty(1, 256, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_gemm_w4a16(X, codes, scales, None, 256, 128, True, Y, None)
+    assert e.value.status == wq.WQ_ERR_WORKSPACE
+
+
 def test_deterministic():
     wl = WORKLOADS["7b-decode"]
     W = wl.weight(1)
