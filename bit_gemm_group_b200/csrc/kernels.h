@@ -21,6 +21,9 @@ int launch_gemv_w4a16_tc(const void* X, int64_t M, int64_t K, const void* codes,
                          const void* scales, const void* zeros, int64_t N, int sym, void* Y,
                          void* ws, cudaStream_t s);
 size_t gemv_workspace_bytes(int64_t N, int64_t K);
+int launch_gemm_w4a16(const void* X, int64_t M, int64_t K, const void* codes,
+                      const void* scales, const void* zeros, int64_t N, int sym, void* Y,
+                      cudaStream_t s);
 
 int launch_gemm_w8a8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
                      int64_t N, void* Y, void* ws, void* acc_out, cudaStream_t s);

@@ -179,7 +179,7 @@ int wq_gemm_w4a16(const void* X, int64_t M, int64_t K, const void* codes, const 
     return wq_host::launch_gemv_w4a16_tc(X, M, K, codes, scales, zeros, N, sym, Y, ws,
                                          as_stream(stream));
   }
-  return WQ_ERR_UNSUPPORTED;
+  return wq_host::launch_gemm_w4a16(X, M, K, codes, scales, zeros, N, sym, Y, as_stream(stream));
 }
 
 int wq_quant_act_i8(const void* X, int64_t M, int64_t K, void* q, void* s, void* stream) {
