@@ -169,6 +169,22 @@ def flush_l2(buf):
     buf.add_(1)
 
 
+def time_flushed(fn, flush, reps=10, warm=3):
+    """Median device time (ms) of fn() with the L2 flushed before each run."""
+    for _ in range(warm):
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts)
+
+
 # ----------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -345,6 +361,51 @@ def secondary(wq, dev, args):
         b = sum(decode_bytes(s["N"], s["K"], M) for s in sets)
         out[f"decode_M{M}_gbs"] = round(b / (tot_ms * 1e-3) / 1e9, 1)
         del sets
+    torch.cuda.empty_cache()
+
+    # 70B decode shapes at M = 1 (asymmetric, fp16 scale + zero), 3 rotating copies
+    wl70 = WORKLOADS["70b-decode"]
+    sets = setup_decode(wq, wl70, 1, dev, 3)
+    tot_ms = 0.0
+    for s in sets:
+        g = capture_shape_graph(wq, s, False, 3, 0)
+        tot_ms += time_graph(g, 10) / 3
+    b = sum(decode_bytes(s["N"], s["K"], 1, asym=True) for s in sets)
+    out["decode_70b_M1_gbs"] = round(b / (tot_ms * 1e-3) / 1e9, 1)
+    del sets
+    torch.cuda.empty_cache()
+
+    # prefill W4A16 GEMM, X [2048, 4096] x W [11008, 4096]^T (L2 flushed between runs)
+    wlp = WORKLOADS["prefill"]
+    Wp = wlp.weight(0).to(dev)
+    N, K = Wp.shape
+    codes, scales, _ = wq.quantize_pack(Wp, 128, 4, True)
+    del Wp
+    Xp = wlp.activation(2048, K).to(dev)
+    Yp = torch.empty((2048, N), dtype=torch.bfloat16, device=dev)
+    t = time_flushed(lambda: wq.wq_gemm_w4a16(Xp, codes, scales, None, N, 128, True, Yp), flush)
+    flops = 2.0 * 2048 * N * K
+    out["prefill_w4a16_tflops"] = round(flops / (t * 1e-3) / 1e12, 1)
+    out["prefill_w4a16_us"] = round(t * 1e3, 1)
+    out["prefill_frac_bf16_peak"] = round(flops / (t * 1e-3) / 1e12 / pk["bf16_tflops"], 3)
+    del codes, scales, Xp, Yp
+
+    # W8A8: per-token act quant + int8 tensor-core GEMM, 4096^3
+    wl8 = WORKLOADS["w8a8"]
+    W8 = wl8.weight(0).to(dev)
+    qw, sw, _ = wq.quantize_pack(W8, W8.shape[1], 8, True)
+    del W8
+    X8 = wl8.activation(4096, 4096).to(dev)
+    Y8 = torch.empty((4096, 4096), dtype=torch.bfloat16, device=dev)
+    ws8 = torch.empty((wq.wq_w8a8_workspace_bytes(4096, 4096),), dtype=torch.uint8, device=dev)
+    t = time_flushed(lambda: wq.wq_gemm_w8a8(X8, qw, sw, Y8, ws8), flush)
+    ops = 2.0 * 4096 ** 3
+    int8_peak = 2.0 * pk["bf16_tflops"]  # measured bf16 peak x the nominal int8/bf16 ratio
+    out["w8a8_tops"] = round(ops / (t * 1e-3) / 1e12, 1)
+    out["w8a8_us"] = round(t * 1e3, 1)
+    out["w8a8_frac_int8_peak"] = round(ops / (t * 1e-3) / 1e12 / int8_peak, 3)
+    out["int8_peak_tops"] = int8_peak
+    del qw, sw, X8, Y8, ws8
     torch.cuda.empty_cache()
     return out
 
