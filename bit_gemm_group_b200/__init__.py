@@ -38,6 +38,7 @@ EXPORTED = (
     "wq_quant_act_i8",
     "wq_w8a8_workspace_bytes", "wq_gemm_w8a8", "wq_get_device_status",
     "wq_status_str", "wq_last_cuda_error", "wq_selftest_wait_timeout",
+    "wq_gemm_w4a16_noalloc",
 )
 
 
@@ -92,6 +93,8 @@ def _declare(L):
     L.wq_get_device_status.argtypes = [_P, _INT]
     L.wq_status_str.argtypes = [_INT]
     L.wq_status_str.restype = ctypes.c_char_p
+    L.wq_gemm_w4a16_noalloc.argtypes = [_P, _I64, _I64, _P, _P, _P, _I64, _INT, _INT, _P, _P]
+    L.wq_gemm_w4a16_noalloc.restype = _INT
     L.wq_selftest_wait_timeout.argtypes = [_INT, _P]
     L.wq_selftest_wait_timeout.restype = _INT
     L.wq_last_cuda_error.argtypes = []
@@ -161,6 +164,16 @@ def wq_gemm_w4a16(X, codes, scales, zeros, N, group_size, sym, Y, ws=None, strea
                              group_size, int(bool(sym)), _ptr(Y), _ptr(ws), ws_bytes,
                              _stream(stream))
     _check(st, "wq_gemm_w4a16")
+
+
+def wq_gemm_w4a16_noalloc(X, codes, scales, zeros, N, group_size, sym, Y, stream=None):
+    """Decode product (M <= 16) on library-owned scratch: no workspace, no
+    allocation.  Overlapping calls race; the first call per device must not
+    be inside a stream capture."""
+    M, K = X.shape
+    st = lib().wq_gemm_w4a16_noalloc(_ptr(X), M, K, _ptr(codes), _ptr(scales), _ptr(zeros), N,
+                                     group_size, int(bool(sym)), _ptr(Y), _stream(stream))
+    _check(st, "wq_gemm_w4a16_noalloc")
 
 
 def wq_quant_act_i8(X, q, s, stream=None):

@@ -35,6 +35,8 @@
 // accumulation is fp32.
 #include <stdlib.h>
 
+#include <mutex>
+
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -513,3 +515,73 @@ int launch_gemv_w4a16_tc(const void* X, int64_t M, int64_t K, const void* codes,
 }
 
 }  // namespace wq_host
+
+// ---------------------------------------------------------------------------
+// Decode product without any allocation
+// ---------------------------------------------------------------------------
+// wq_gemm_w4a16 asks its caller for a small workspace (per-tile arrival
+// counters and per-CTA partial sums of the split tiles).  Some callers cannot
+// provide one: code that runs while a CUDA graph is being captured must not
+// call cudaMalloc, a serving loop may run under a fixed memory budget owned by
+// another allocator, and plain C hosts may have no allocator hooked to the
+// device at all.  wq_gemm_w4a16_noalloc runs the same kernel on scratch that
+// lives in this library's own device image: a file-scope array that every GPU
+// which loads the library holds until the process exits.
+namespace {
+constexpr int64_t kNoAllocMaxN = 131072;   // 1024 row tiles of 128
+constexpr int64_t kNoAllocMaxCtas = 256;   // one CTA per SM, up to 256 SMs
+constexpr size_t kNoAllocCntBytes = size_t(kNoAllocMaxN / 128) * 4;                   // 4 KiB
+constexpr size_t kNoAllocPartBytes = size_t(kNoAllocMaxCtas) * 2 * 128 * 16 * 4;     // 4 MiB
+constexpr size_t kNoAllocBytes = kNoAllocCntBytes + kNoAllocPartBytes;
+}  // namespace
+
+// The scratch itself.  Its name, used in host code, is only a host-side
+// stand-in for the symbol: the device address comes from
+// cudaGetSymbolAddress, taken once per device with that device current.
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocBytes];
+
+namespace {
+void* g_noalloc_ptr[64] = {};
+std::mutex g_noalloc_mu;
+}  // namespace
+
+extern "C" int wq_gemm_w4a16_noalloc(const void* X, int64_t M, int64_t K, const void* codes,
+                                     const void* scales, const void* zeros, int64_t N,
+                                     int group_size, int sym, void* Y, void* stream) {
+  if (M < 0 || K < 0 || N < 0) return WQ_ERR_ARG;
+  if (sym != 0 && sym != 1) return WQ_ERR_ARG;
+  if ((sym == 1) != (zeros == nullptr)) return WQ_ERR_ARG;
+  if (group_size != 128) return WQ_ERR_UNSUPPORTED;
+  if ((K % 128) != 0 || (N % 8) != 0) return WQ_ERR_ALIGN;
+  if (M > 16 || N > kNoAllocMaxN || K > (int64_t(1) << 24)) return WQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return WQ_OK;
+  if (K == 0) return WQ_ERR_ARG;
+  if (!X || !codes || !scales || !Y) return WQ_ERR_ARG;
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!a16(X) || !a16(codes) || !a16(scales) || !a16(Y) || (zeros && !a16(zeros)))
+    return WQ_ERR_ALIGN;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  int dev = 0;
+  WQ_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev >= 64) return WQ_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  {
+    // set-up on the first call for this device (this device is current)
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      WQ_CUDA_CHECK(cudaGetSymbolAddress(&p, g_decode_scratch));
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  if (int64_t(wq_host::sm_count()) > kNoAllocMaxCtas ||
+      wq_host::gemv_workspace_bytes(N, K) > kNoAllocBytes)
+    return WQ_ERR_UNSUPPORTED;
+  // the arrival counters must start at zero: clear them on the call's stream
+  const size_t cnt = (size_t((N + 127) / 128) * 4 + 255) & ~size_t(255);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WQ_CUDA_CHECK(cudaMemsetAsync(scratch, 0, cnt, s));
+  return wq_host::launch_gemv_w4a16_tc(X, M, K, codes, scales, zeros, N, sym, Y, scratch, s);
+}

@@ -132,6 +132,29 @@ WQ_API int wq_gemm_w4a16(const void *X, int64_t M, int64_t K, const void *codes,
                          size_t ws_bytes, void *stream);
 
 /*
+ * wq_gemm_w4a16_noalloc -- the decode product of wq_gemm_w4a16 (M = 1..16)
+ * for callers that cannot allocate device memory: code running while a CUDA
+ * graph is being captured (cudaMalloc is not allowed there), serving loops
+ * whose device memory belongs to another allocator, C hosts without a device
+ * allocator.  The quantization write-ups have no counterpart of this call.
+ *
+ * Same arguments and results as wq_gemm_w4a16 without ws / ws_bytes.  The
+ * library allocates nothing, in this call or ever: the scratch is an array of
+ * 4 MiB + 4 KiB inside the library's device image, held by every GPU that
+ * loads the library until the process exits.  Limits: M <= 16, N <= 131072,
+ * at most 256 SMs (WQ_ERR_UNSUPPORTED beyond them).
+ *
+ * The first call on a device looks up the array's device address; make that
+ * first call before any stream capture.  Every call shares the one array and
+ * clears its counters on its own stream: calls that overlap on the GPU (other
+ * streams, other host threads) race and give wrong results -- serialize them.
+ */
+WQ_API int wq_gemm_w4a16_noalloc(const void *X, int64_t M, int64_t K,
+                                 const void *codes, const void *scales,
+                                 const void *zeros, int64_t N, int group_size,
+                                 int sym, void *Y, void *stream);
+
+/*
  * wq_quant_act_i8 -- per-token dynamic INT8 quantization of activations
  * ([P4] sec. 6 per-token absmax quantizer, used for the A8 of W8A8, [P4]
  * sec. 2.3): s[m] = max(amax_m / 127, 1e-8); q = clamp(round(x / s), -128, 127).
