@@ -491,6 +491,45 @@ def run_reference(args, rank, world, budget_s=60.0):
     print(json.dumps(line), flush=True)
 
 
+def profile_case(case):
+    """Three launches of one kernel on its workload, nothing else timed:
+    decode = W4A16 decode product on [11008, 4096] at M = 1, prefill = W4A16
+    GEMM 2048 x 11008 x 4096, w8a8 = W8A8 GEMM 4096^3."""
+    import bit_gemm_group_b200 as wq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if case == "decode":
+        wl = WORKLOADS["7b-decode"]
+        W = wl.weight(1).to(dev)
+        N, K = W.shape
+        c, s, z = wq.quantize_pack(W, 128, 4, True)
+        X = wl.activation(1, K).to(dev)
+        Y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+        ws = wq.w4a16_workspace(1, N, K, dev)
+        for _ in range(3):
+            wq.wq_gemm_w4a16(X, c, s, None, N, 128, True, Y, ws)
+    elif case == "prefill":
+        wl = WORKLOADS["prefill"]
+        W = wl.weight(0).to(dev)
+        N, K = W.shape
+        c, s, z = wq.quantize_pack(W, 128, 4, True)
+        X = wl.activation(2048, K).to(dev)
+        Y = torch.empty((2048, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            wq.wq_gemm_w4a16(X, c, s, None, N, 128, True, Y)
+    else:
+        wl = WORKLOADS["w8a8"]
+        W = wl.weight(0).to(dev)
+        qw, sw, _ = wq.quantize_pack(W, W.shape[1], 8, True)
+        X = wl.activation(4096, 4096).to(dev)
+        Y = torch.empty((4096, 4096), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty((wq.wq_w8a8_workspace_bytes(4096, 4096),), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            wq.wq_gemm_w8a8(X, qw, sw, Y, ws)
+    torch.cuda.synchronize()
+    print(case, "status", wq.wq_status_str(wq.wq_get_device_status()))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -499,7 +538,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--quick", action="store_true", help="skip the secondary rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
+    ap.add_argument("--profile-case", choices=["decode", "prefill", "w8a8"],
+                    help="run one kernel 3 times on its workload (for ncu captures) and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

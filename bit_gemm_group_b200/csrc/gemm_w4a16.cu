@@ -204,18 +204,29 @@ __global__ void __launch_bounds__(THREADS, 1)
     st.advance(STAGES, w);
     ab.advance(NA, w);
     bool ok = true;
-    int gi = 0;  // global stage index of this CTA (all tiles); ours: gi % NDQ == w
+    int gi = 0;  // global index of the tile's first stage; ours: index % NDQ == w
     for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
       const int wt = tile / XT;
       const int n = wt * BW + row;
       const bool row_in = n < N;
       const __half* srow = scales + size_t(row_in ? n : 0) * G;
       const __half* zrow = sym ? nullptr : zeros + size_t(row_in ? n : 0) * G;
-      for (int kb = 0; kb < KB; ++kb, ++gi) {
-        if (gi % NDQ != w) continue;
-        const int g = kb >> 1;  // two stages per 128-wide group
-        const float s = row_in ? __half2float(srow[g]) : 0.f;
-        const float zf = sym ? 8.f : (row_in ? __half2float(zrow[g]) : 0.f);
+      // this warpgroup's first stage of the tile and its group's scale / zero;
+      // each iteration fetches the next stage's pair before working, so the
+      // loads have a whole stage of work to land
+      int kb = (w - gi % NDQ + NDQ) % NDQ;
+      float s_nx = 0.f, z_nx = 8.f;
+      if (kb < KB && row_in) {
+        s_nx = __half2float(srow[kb >> 1]);
+        if (!sym) z_nx = __half2float(zrow[kb >> 1]);
+      }
+      for (; kb < KB; kb += NDQ) {
+        const float s = s_nx, zf = sym ? 8.f : z_nx;
+        if (kb + NDQ < KB && row_in) {
+          const int gn = (kb + NDQ) >> 1;  // two stages per 128-wide group
+          s_nx = __half2float(srow[gn]);
+          if (!sym) z_nx = __half2float(zrow[gn]);
+        }
         if (!(ok = tc::wait_bounded(&sm.full[st.slot], st.phase, wd) &&
                    tc::wait_bounded(&sm.a_empty[ab.slot], ab.phase ^ 1u, wd)))
           break;
@@ -247,6 +258,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         st.advance(STAGES, NDQ);
         ab.advance(NA, NDQ);
       }
+      gi += KB;
     }
   } else if (warp >= EPI_WARP0) {
     // ------------------------------------------------------------ epilogue
