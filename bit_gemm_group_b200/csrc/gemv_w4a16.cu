@@ -514,6 +514,25 @@ int launch_gemv_w4a16_tc(const void* X, int64_t M, int64_t K, const void* codes,
   return WQ_OK;
 }
 
+// One workspace size for every M <= 16 (the CUDA-core kernel needs none), so
+// a caller's workspace serves both decode kernels.
+size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  (void)M;
+  return gemv_workspace_bytes(N, K);
+}
+
+bool decode_on_cuda_cores(int64_t M, int64_t K) {
+  return M <= kGemvCcMaxM && gemv_cc_depth(M, K) > 0;
+}
+
+int launch_decode_w4a16(const void* X, int64_t M, int64_t K, const void* codes,
+                        const void* scales, const void* zeros, int64_t N, int sym, void* Y,
+                        void* ws, cudaStream_t s) {
+  if (decode_on_cuda_cores(M, K))
+    return launch_gemv_w4a16_cc(X, M, K, codes, scales, zeros, N, sym, Y, s);
+  return launch_gemv_w4a16_tc(X, M, K, codes, scales, zeros, N, sym, Y, ws, s);
+}
+
 }  // namespace wq_host
 
 // ---------------------------------------------------------------------------
@@ -576,12 +595,14 @@ extern "C" int wq_gemm_w4a16_noalloc(const void* X, int64_t M, int64_t K, const 
     }
     scratch = g_noalloc_ptr[dev];
   }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (wq_host::decode_on_cuda_cores(M, K))  // no scratch at all
+    return wq_host::launch_gemv_w4a16_cc(X, M, K, codes, scales, zeros, N, sym, Y, s);
   if (int64_t(wq_host::sm_count()) > kNoAllocMaxCtas ||
       wq_host::gemv_workspace_bytes(N, K) > kNoAllocBytes)
     return WQ_ERR_UNSUPPORTED;
   // the arrival counters must start at zero: clear them on the call's stream
   const size_t cnt = (size_t((N + 127) / 128) * 4 + 255) & ~size_t(255);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   WQ_CUDA_CHECK(cudaMemsetAsync(scratch, 0, cnt, s));
   return wq_host::launch_gemv_w4a16_tc(X, M, K, codes, scales, zeros, N, sym, Y, scratch, s);
 }

@@ -154,7 +154,7 @@ int wq_dequant(const void* codes, const void* scales, const void* zeros, int64_t
 size_t wq_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || M > 16 || N <= 0 || K < 128) return 0;
   if (wq_host::ensure_device() != WQ_OK) return 0;
-  return wq_host::gemv_workspace_bytes(N, K);
+  return wq_host::decode_workspace_bytes(M, N, K);
 }
 
 int wq_gemm_w4a16(const void* X, int64_t M, int64_t K, const void* codes, const void* scales,
@@ -175,9 +175,9 @@ int wq_gemm_w4a16(const void* X, int64_t M, int64_t K, const void* codes, const 
   int st = wq_host::ensure_device();
   if (st != WQ_OK) return st;
   if (M <= 16) {
-    if (!ws || ws_bytes < wq_host::gemv_workspace_bytes(N, K)) return WQ_ERR_WORKSPACE;
-    return wq_host::launch_gemv_w4a16_tc(X, M, K, codes, scales, zeros, N, sym, Y, ws,
-                                         as_stream(stream));
+    if (!ws || ws_bytes < wq_host::decode_workspace_bytes(M, N, K)) return WQ_ERR_WORKSPACE;
+    return wq_host::launch_decode_w4a16(X, M, K, codes, scales, zeros, N, sym, Y, ws,
+                                        as_stream(stream));
   }
   return wq_host::launch_gemm_w4a16(X, M, K, codes, scales, zeros, N, sym, Y, as_stream(stream));
 }

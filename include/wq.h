@@ -114,14 +114,19 @@ WQ_API int wq_dequant(const void *codes, const void *scales, const void *zeros,
  * to memory).  X bf16 [M, K]; codes/scales/zeros as above with
  * group_size == 128 (others: WQ_ERR_UNSUPPORTED, [P4] sec. 7.2: the group must
  * divide the kernel tile); Y bf16 [M, N]; fp32 accumulation.
- * M <= 16 runs the decode kernel (every weight byte streamed once from HBM,
- * the work split evenly over all SMs); larger M runs the tensor-core GEMM.
+ * M <= 16 runs a decode kernel (every weight byte streamed once from HBM,
+ * the work split evenly over all SMs): M <= 2 on the CUDA cores while the
+ * prepared X (two int8 limbs per element) fits in shared memory, i.e.
+ * K <= 76800 at M = 1 and K <= 37888 at M = 2, else on the tensor cores;
+ * larger M runs the tensor-core GEMM.
  * Requires K % 128 == 0 and N % 8 == 0.
  *
  * ws / ws_bytes: device workspace of wq_w4a16_workspace_bytes(M, N, K) bytes
  * (0 for M > 16, where ws may be NULL).  Fill it with zeros once before its
- * first use (e.g. cudaMemset); every call that completes leaves it zeroed
- * again, so it can be reused call after call.  Calls that may run at the same
+ * first use (e.g. cudaMemset); every call that completes leaves the part that
+ * must start at zero (the arrival counters at its start) zeroed again, so it
+ * can be reused call after call (its size does not depend on M).  The
+ * CUDA-core kernel does not use it.  Calls that may run at the same
  * time on the GPU need separate workspaces.  After a call reported
  * WQ_ERR_TIMEOUT, zero it again.  WQ_ERR_WORKSPACE if NULL or too small.
  */

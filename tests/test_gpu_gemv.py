@@ -76,6 +76,30 @@ def test_ragged(M, N, K, sym):
     check_gemv(make_activation(M, K, seed=M), dq, oq, sym, rounding_aware=N < 256)
 
 
+@pytest.mark.parametrize("kind", ["positive", "outlier_dims", "row_scales", "sparse_groups"])
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_activation_structure(kind, M):
+    """Activation value structure that stresses the per-(group, row) handling:
+    all-positive values (large same-sign sums), outlier hidden dims of
+    magnitude 50-100, rows whose magnitudes differ by 10^6, and groups that
+    are entirely zero."""
+    N, K = 4096, 4096
+    W = make_weight(N, K, 0.02, seed=11, outlier_frac=0.001, outlier_scale=30.0)
+    dq, oq = quantized(W, False)
+    if kind == "outlier_dims":
+        X = make_activation(M, K, seed=M, outlier_dims=6)
+    else:
+        X = make_activation(M, K, seed=M).float()
+        if kind == "positive":
+            X = X.abs() + 0.5
+        elif kind == "row_scales":
+            X = X * torch.logspace(-3, 3, M).reshape(M, 1) if M > 1 else X * 1e-3
+        else:
+            X.view(M, K // 128, 128)[:, 1::3, :] = 0.0
+        X = X.to(torch.bfloat16)
+    check_gemv(X, dq, oq, False)
+
+
 def test_workspace_reused_and_left_zeroed():
     W = make_weight(1000 * 8, 4096, 0.02, seed=3)
     dq, oq = quantized(W, True)
@@ -88,6 +112,22 @@ def test_workspace_reused_and_left_zeroed():
     assert int(ws[: 4 * T].count_nonzero()) == 0  # arrival counters reset by every call
 
 
+def test_workspace_shared_by_both_decode_kernels():
+    """One workspace, sized for the largest request, serves the CUDA-core
+    kernel (M <= 2) and the tensor-core kernel (M = 3..16) alternately."""
+    N, K = 4096, 4096
+    W = make_weight(N, K, 0.02, seed=5)
+    (codes, scales, zeros), _ = quantized(W, False)
+    Xs = {M: make_activation(M, K, seed=M).cuda() for M in (1, 2, 4, 16)}
+    ref = {M: wq.gemm_w4a16(X, codes, scales, zeros, 128, False) for M, X in Xs.items()}
+    nbytes = max(wq.lib().wq_w4a16_workspace_bytes(M, N, K) for M in Xs)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    for M in (1, 4, 2, 16, 1, 4):
+        Y = wq.gemm_w4a16(Xs[M], codes, scales, zeros, 128, False, ws=ws)
+        assert torch.equal(Y, ref[M]), M
+    assert int(ws[: 4 * (N // 128)].count_nonzero()) == 0
+
+
 def test_workspace_too_small():
     W = make_weight(256, 1024, 0.02, seed=3).cuda()
     codes, scales, _ = wq.quantize_pack(W, 128, 4, True)
@@ -98,11 +138,12 @@ def test_workspace_too_small():
     assert e.value.status == wq.WQ_ERR_WORKSPACE
 
 
-def test_deterministic():
+@pytest.mark.parametrize("M", [1, 2, 4])
+def test_deterministic(M):
     wl = WORKLOADS["7b-decode"]
     W = wl.weight(1)
     (codes, scales, zeros), _ = quantized(W, True)
-    X = wl.activation(4, W.shape[1]).cuda()
+    X = wl.activation(M, W.shape[1]).cuda()
     a = wq.gemm_w4a16(X, codes, scales, zeros)
     b = wq.gemm_w4a16(X, codes, scales, zeros)
     assert torch.equal(a, b)
