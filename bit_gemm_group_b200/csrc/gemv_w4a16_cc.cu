@@ -294,6 +294,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_cc_kernel(
   Pos cur{rb0 + int(s0 / sh.C), int(s0 % sh.C)};
   const int b_first = cur.b;
 
+  // A kernel launched right after this one may be scheduled as soon as SMs
+  // free up; it only prefetches weights until this grid has finished.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // the warp's first D items go out before anything else
   Pos ahead = cur;
 #pragma unroll
@@ -307,6 +310,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_cc_kernel(
   szp.next(sh.C);
   load_sz(v1, scales, zeros, szp, 1 < n_it, sh, lane);
   szp.next(sh.C);
+  // X may be the previous kernel's output, and Y its input: wait for that
+  // grid (when launched as its dependent) before touching either
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   prepare_x(X, sh.M, sh.K, sh.C, xs, sx, invs);
   __syncthreads();
 
@@ -404,9 +410,20 @@ static cudaError_t launch_cc(dim3 grid, size_t smem, cudaStream_t s, const __nv_
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-  wq::gemv_cc::gemv_cc_kernel<MT, D><<<grid, wq::gemv_cc::THREADS, smem, s>>>(X, codes, scales,
-                                                                              zeros, Y, sh);
-  return cudaGetLastError();
+  // programmatic dependent launch: the weight prefetch of this kernel
+  // overlaps the tail of the kernel before it on the stream
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(wq::gemv_cc::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, wq::gemv_cc::gemv_cc_kernel<MT, D>, X, codes, scales, zeros, Y,
+                            sh);
 }
 
 int launch_gemv_w4a16_cc(const void* X, int64_t M, int64_t K, const void* codes,
