@@ -158,38 +158,59 @@ struct Pos {
 };
 
 // Copies the codes of the item at p (when `live`) into ring slot `slot` and
-// closes one cp.async group (an empty one otherwise).
+// closes one cp.async group (an empty one otherwise).  Items whose R rows all
+// exist take the path without per-row checks.
 __device__ __forceinline__ void issue_item(uint4* __restrict__ ring_w, int slot,
                                            const uint8_t* __restrict__ codes, Pos p, bool live,
                                            const Shape& sh, int lane) {
   const int k = p.c * CHUNK + lane * 32;
   if (live && k < sh.K) {
+    const size_t rowb = size_t(sh.K >> 1);
+    const uint8_t* src = codes + size_t(p.b * R) * rowb + (k >> 1);
+    uint4* dst = ring_w + slot * (R * 32) + lane;
+    if (p.b * R + R <= sh.N) {
 #pragma unroll
-    for (int r = 0; r < R; ++r)
-      if (p.b * R + r < sh.N)
-        cp_async16(ring_w + (slot * R + r) * 32 + lane,
-                   codes + size_t(p.b * R + r) * size_t(sh.K >> 1) + (k >> 1));
+      for (int r = 0; r < R; ++r) cp_async16(dst + r * 32, src + r * rowb);
+    } else {
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        if (p.b * R + r < sh.N) cp_async16(dst + r * 32, src + r * rowb);
+    }
   }
   cp_async_commit();
 }
 
-// Scales and zero points of one item for its R rows.
+// Scales (as fp32) and zero points (as integers) of one item for its R rows.
 struct ItemSZ {
-  __half s[R];
-  __half z[R];  // integer values 0..15
+  float s[R];
+  int z[R];
 };
 
+// Loads v for the item at p when `live` (a lane past K, or a row past N,
+// keeps what it had: its values are never used).  Zero points are loaded only
+// for asymmetric weights; symmetric ones keep z = 8.
 __device__ __forceinline__ void load_sz(ItemSZ& v, const __half* __restrict__ scales,
                                         const __half* __restrict__ zeros, Pos p, bool live,
                                         const Shape& sh, int lane) {
-  const __half h0 = __ushort_as_half(0), h8 = __ushort_as_half(0x4800);  // 0, 8
   const int k = p.c * CHUNK + lane * 32;
+  if (!live || k >= sh.K) return;
+  const size_t gi = size_t(p.b * R) * size_t(sh.G) + (k >> 7);
+  const __half* sp = scales + gi;
+  const __half* zp = zeros + gi;
+  if (p.b * R + R <= sh.N) {
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const bool ok = live && k < sh.K && p.b * R + r < sh.N;
-    const size_t gi = ok ? size_t(p.b * R + r) * size_t(sh.G) + (k >> 7) : 0;
-    v.s[r] = ok ? scales[gi] : h0;
-    v.z[r] = sh.sym ? h8 : (ok ? zeros[gi] : h0);
+    for (int r = 0; r < R; ++r) v.s[r] = __half2float(__ldg(sp + r * sh.G));
+    if (!sh.sym) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) v.z[r] = __half2int_rn(__ldg(zp + r * sh.G));
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (p.b * R + r < sh.N) {
+        v.s[r] = __half2float(__ldg(sp + r * sh.G));
+        if (!sh.sym) v.z[r] = __half2int_rn(__ldg(zp + r * sh.G));
+      }
   }
 }
 
@@ -236,8 +257,8 @@ __device__ __forceinline__ void compute_item(const uint4* __restrict__ words, co
       const float fi = invs[m * sh.G + g];
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        const int t = ah[r][m] * 128 + al[r][m] - int(__half2float(v.z[r])) * sxl;  // exact
-        acc[r][m] = fmaf(float(t), __half2float(v.s[r]) * fi, acc[r][m]);
+        const int t = ah[r][m] * 128 + al[r][m] - v.z[r] * sxl;  // exact
+        acc[r][m] = fmaf(float(t), v.s[r] * fi, acc[r][m]);
       }
     }
   }
@@ -304,11 +325,17 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_cc_kernel(
     issue_item(ring_w, d, codes, ahead, d < n_it, sh, lane);
     ahead.next(sh.C);
   }
-  ItemSZ v0, v1;
+  // scales and zero points run two items ahead, in two alternating sets
+  ItemSZ va, vb;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    va.s[r] = vb.s[r] = 0.f;
+    va.z[r] = vb.z[r] = 8;
+  }
   Pos szp = cur;
-  load_sz(v0, scales, zeros, szp, 0 < n_it, sh, lane);
+  load_sz(va, scales, zeros, szp, 0 < n_it, sh, lane);
   szp.next(sh.C);
-  load_sz(v1, scales, zeros, szp, 1 < n_it, sh, lane);
+  load_sz(vb, scales, zeros, szp, 1 < n_it, sh, lane);
   szp.next(sh.C);
   // X may be the previous kernel's output, and Y its input: wait for that
   // grid (when launched as its dependent) before touching either
@@ -324,15 +351,16 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_cc_kernel(
   float* part_w = part + warp * (2 * R * MT_MAX);
   int slot = 0;
   int c_start = cur.c;  // first chunk of the current row block this warp holds
-  for (int it = 0; it < n_it; ++it) {
+  // one item: compute it from the ring and `v`, refill its slot with the item
+  // D ahead, load `v` for the item two ahead, emit finished row blocks
+  auto step = [&](ItemSZ& v, int it) {
     cp_async_wait<D - 1>();  // this lane's copies of item `it` have landed
-    compute_item<MT>(ring_w + slot * R * 32 + lane, v0, acc, xs, sx, invs, cur.c, sh, lane);
+    compute_item<MT>(ring_w + slot * R * 32 + lane, v, acc, xs, sx, invs, cur.c, sh, lane);
     // refill the slot just read (its words are in registers) with item it + D
     issue_item(ring_w, slot, codes, ahead, it + D < n_it, sh, lane);
     ahead.next(sh.C);
     slot = (slot + 1 == D) ? 0 : slot + 1;
-    v0 = v1;
-    load_sz(v1, scales, zeros, szp, it + 2 < n_it, sh, lane);
+    load_sz(v, scales, zeros, szp, it + 2 < n_it, sh, lane);
     szp.next(sh.C);
     if (cur.c == sh.C - 1 || it + 1 == n_it) {
       emit_block<MT>(acc, cur.b, c_start == 0 && cur.c == sh.C - 1, cur.b == b_first ? 0 : 1,
@@ -340,6 +368,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_cc_kernel(
       c_start = 0;
     }
     cur.next(sh.C);
+  };
+  for (int it = 0; it < n_it; it += 2) {
+    step(va, it);
+    if (it + 1 == n_it) break;
+    step(vb, it + 1);
   }
   cp_async_wait<0>();
   __syncthreads();
