@@ -33,7 +33,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import WORKLOADS, bf16_bits  # noqa: E402
+from workloads import WORKLOADS, bf16_bits, make_activation  # noqa: E402
 
 METRIC = "W4A16-g128 dequant-GEMM: HBM GB/s at M=1, TFLOPS at M=2048, % of roofline"
 ROT = 10  # rotating weight copies (10 x 55 MB = 550 MB > 4 x 126 MB L2)
@@ -151,6 +151,31 @@ def capture_shape_graph(wq, s, sym, count, start):
                 wq.wq_gemm_w4a16(s["X"], c, sc, z, s["N"], 128, sym, s["Y"], s["ws"])
     torch.cuda.current_stream().wait_stream(stream)
     return g
+
+
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemv_cc_kernel_7b_decode_step.txt")
+DECODE_SRC = os.path.join(ROOT, "bit_gemm_group_b200", "csrc", "gemv_w4a16_cc.cu")
+
+
+def recorded_traffic():
+    """DRAM bytes (read + write) of one 7B decode step (its three decode
+    launches) from the committed ncu capture, or None when the decode kernel's
+    source has changed since that capture (or there is none)."""
+    import hashlib
+    try:
+        fields = {}
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                if ":" in line:
+                    k, v = line.split(":", 1)
+                    fields[k.strip()] = v.strip()
+        with open(DECODE_SRC, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        if fields.get("kernel_source_sha256") != sha:
+            return None
+        return int(fields["dram_bytes_per_step"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def time_graph(g, reps):
@@ -275,7 +300,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2) if achieved else None,
                      "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / pk["hbm_gbs"], 4) if achieved else None,
-                     "traffic": None, "kernel": "wq W4A16 decode product",
+                     "traffic": recorded_traffic(), "traffic_unit": "bytes per step",
+                     "kernel": "wq W4A16 decode product",
                      "peak_source": pk["source"],
                      "per_shape_us": [round(1e3 * k / max(1, launches_timed), 3)
                                       for k in kern_ms]},
@@ -492,13 +518,40 @@ def run_reference(args, rank, world, budget_s=60.0):
 
 
 def profile_case(case):
-    """Three launches of one kernel on its workload, nothing else timed:
-    decode = W4A16 decode product on [11008, 4096] at M = 1, prefill = W4A16
-    GEMM 2048 x 11008 x 4096, w8a8 = W8A8 GEMM 4096^3."""
+    """Launches of one kernel on its workload, nothing else timed:
+    decode = W4A16 decode product on [11008, 4096] at M = 1 (three launches),
+    decode-large = the same on [57344, 8192] (a fused gate/up projection of a
+    70B model, 235 MB of codes, larger than L2; three launches), decode-step =
+    two warm-up steps then one step of the 7B decode workload (its three
+    shapes), prefill = W4A16 GEMM 2048 x 11008 x 4096, w8a8 = W8A8 GEMM 4096^3
+    (three launches each)."""
     import bit_gemm_group_b200 as wq
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    if case == "decode":
+    if case == "decode-large":
+        N, K = 57344, 8192
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(7)
+        W = (torch.randn((N, K), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+        c, s, z = wq.quantize_pack(W, 128, 4, True)
+        del W
+        X = make_activation(1, K, seed=7).to(dev)
+        Y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+        ws = wq.w4a16_workspace(1, N, K, dev)
+        for _ in range(3):
+            wq.wq_gemm_w4a16(X, c, s, None, N, 128, True, Y, ws)
+    elif case == "decode-step":
+        wl = WORKLOADS["7b-decode"]
+        sets = []
+        for i, (N, K) in enumerate(wl.shapes):
+            c, s, z = wq.quantize_pack(wl.weight(i).to(dev), 128, 4, True)
+            sets.append((N, K, c, s, wl.activation(1, K).to(dev),
+                         torch.empty((1, N), dtype=torch.bfloat16, device=dev),
+                         wq.w4a16_workspace(1, N, K, dev)))
+        for _ in range(3):
+            for N, K, c, s, X, Y, ws in sets:
+                wq.wq_gemm_w4a16(X, c, s, None, N, 128, True, Y, ws)
+    elif case == "decode":
         wl = WORKLOADS["7b-decode"]
         W = wl.weight(1).to(dev)
         N, K = W.shape
@@ -538,7 +591,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--quick", action="store_true", help="skip the secondary rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
-    ap.add_argument("--profile-case", choices=["decode", "prefill", "w8a8"],
+    ap.add_argument("--profile-case",
+                    choices=["decode", "decode-large", "decode-step", "prefill", "w8a8"],
                     help="run one kernel 3 times on its workload (for ncu captures) and exit")
     args = ap.parse_args()
     if args.profile_case:

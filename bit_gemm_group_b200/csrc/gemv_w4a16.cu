@@ -521,14 +521,20 @@ size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return gemv_workspace_bytes(N, K);
 }
 
-bool decode_on_cuda_cores(int64_t M, int64_t K) {
-  return M <= kGemvCcMaxM && gemv_cc_depth(M, K) > 0;
+bool decode_on_cuda_cores(int64_t M, int64_t N, int64_t K) {
+  if (M > kGemvCcMaxM || gemv_cc_depth(M, K) == 0) return false;
+  if (M <= 2) return true;
+  // Three or four activation rows cost the CUDA-core kernel about twice the
+  // issue slots of one row: it still wins on small matrices, where the
+  // tensor-core kernel's fixed latency dominates (4096 x 4096: 12 vs 15 us),
+  // and loses on large ones (28672 x 8192: 67 vs 56 us).
+  return K <= 8192 && N * K <= (int64_t(1) << 26);
 }
 
 int launch_decode_w4a16(const void* X, int64_t M, int64_t K, const void* codes,
                         const void* scales, const void* zeros, int64_t N, int sym, void* Y,
                         void* ws, cudaStream_t s) {
-  if (decode_on_cuda_cores(M, K))
+  if (decode_on_cuda_cores(M, N, K))
     return launch_gemv_w4a16_cc(X, M, K, codes, scales, zeros, N, sym, Y, s);
   return launch_gemv_w4a16_tc(X, M, K, codes, scales, zeros, N, sym, Y, ws, s);
 }
@@ -596,7 +602,7 @@ extern "C" int wq_gemm_w4a16_noalloc(const void* X, int64_t M, int64_t K, const 
     scratch = g_noalloc_ptr[dev];
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (wq_host::decode_on_cuda_cores(M, K))  // no scratch at all
+  if (wq_host::decode_on_cuda_cores(M, N, K))  // no scratch at all
     return wq_host::launch_gemv_w4a16_cc(X, M, K, codes, scales, zeros, N, sym, Y, s);
   if (int64_t(wq_host::sm_count()) > kNoAllocMaxCtas ||
       wq_host::gemv_workspace_bytes(N, K) > kNoAllocBytes)

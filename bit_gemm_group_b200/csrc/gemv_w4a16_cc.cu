@@ -1,4 +1,4 @@
-// gemv_w4a16_cc.cu -- W4A16 decode product for one or two activation rows on
+// gemv_w4a16_cc.cu -- W4A16 decode product for one to four activation rows on
 // the CUDA cores.
 //
 //   Y[m, n] = sum_g s[n, g] * sum_{k in g} X[m, k] * (u[n, k] - z[n, g])
@@ -8,7 +8,7 @@
 // bandwidth; sec. 2.3 W4A16; "大模型量化技术定义与主流方案解析" sec. 四: the
 // weight is expanded inside the product and never written back.)
 //
-// At M <= 2 the arithmetic per weight byte is small enough for the CUDA cores,
+// At M <= 4 the arithmetic per weight byte is small enough for the CUDA cores,
 // and a streaming kernel keeps every SM's loads in flight from its first cycle
 // to its last, with none of the tensor-core path's hand-offs between warps.
 //
@@ -55,7 +55,7 @@ constexpr int R = 4;                      // weight rows per item
 constexpr int ITEM_BYTES = R * CHUNK / 2; // codes of one item (2 KB)
 constexpr int MAXD = 6;
 constexpr int SMEM_LIMIT = 227 * 1024;
-constexpr int MT_MAX = 2;
+constexpr int MT_MAX = 4;
 
 // sum of the four byte products a_i * b_i plus c; a unsigned, b signed bytes
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
@@ -233,20 +233,24 @@ __device__ __forceinline__ void compute_item(const uint4* __restrict__ words, co
     for (int m = 0; m < MT; ++m) ah[r][m] = al[r][m] = 0;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    uint4 xq[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m)
-      xq[m] = (m < sh.M) ? xs[(m * sh.C + c) * 128 + q * 32 + lane] : make_uint4(0, 0, 0, 0);
+    uint32_t ev[R], od[R];  // even / odd elements of word q as bytes, per row
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const uint32_t w = q == 0 ? wr[r].x : q == 1 ? wr[r].y : q == 2 ? wr[r].z : wr[r].w;
-      const uint32_t ev = w & 0x0F0F0F0Fu, od = (w >> 4) & 0x0F0F0F0Fu;
+      ev[r] = w & 0x0F0F0F0Fu;
+      od[r] = (w >> 4) & 0x0F0F0F0Fu;
+    }
 #pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        ah[r][m] = dp4a_us(ev, xq[m].x, ah[r][m]);
-        al[r][m] = dp4a_us(ev, xq[m].y, al[r][m]);
-        ah[r][m] = dp4a_us(od, xq[m].z, ah[r][m]);
-        al[r][m] = dp4a_us(od, xq[m].w, al[r][m]);
+    for (int m = 0; m < MT; ++m) {
+      if (m < sh.M) {
+        const uint4 xq = xs[(m * sh.C + c) * 128 + q * 32 + lane];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          ah[r][m] = dp4a_us(ev[r], xq.x, ah[r][m]);
+          al[r][m] = dp4a_us(ev[r], xq.y, al[r][m]);
+          ah[r][m] = dp4a_us(od[r], xq.z, ah[r][m]);
+          al[r][m] = dp4a_us(od[r], xq.w, al[r][m]);
+        }
       }
     }
   }
@@ -483,10 +487,12 @@ int launch_gemv_w4a16_cc(const void* X, int64_t M, int64_t K, const void* codes,
   const uint8_t* cd = static_cast<const uint8_t*>(codes);
   __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y);
   cudaError_t e = cudaErrorInvalidValue;
+  const int mt = M <= 1 ? 1 : M <= 2 ? 2 : 4;  // M = 3 runs the 4-row instance
 #define WQ_CC_CASE(MT_, D_) \
-  if (M == MT_ && D == D_) e = launch_cc<MT_, D_>(grid, smem, s, x, cd, sc, zp, y, sh);
+  if (mt == MT_ && D == D_) e = launch_cc<MT_, D_>(grid, smem, s, x, cd, sc, zp, y, sh);
   WQ_CC_CASE(1, 2) WQ_CC_CASE(1, 3) WQ_CC_CASE(1, 4) WQ_CC_CASE(1, 5) WQ_CC_CASE(1, 6)
   WQ_CC_CASE(2, 2) WQ_CC_CASE(2, 3) WQ_CC_CASE(2, 4) WQ_CC_CASE(2, 5) WQ_CC_CASE(2, 6)
+  WQ_CC_CASE(4, 2) WQ_CC_CASE(4, 3) WQ_CC_CASE(4, 4) WQ_CC_CASE(4, 5) WQ_CC_CASE(4, 6)
 #undef WQ_CC_CASE
   if (e != cudaSuccess) return cuda_fail(e, "gemv_cc_kernel");
   return WQ_OK;

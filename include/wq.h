@@ -115,9 +115,10 @@ WQ_API int wq_dequant(const void *codes, const void *scales, const void *zeros,
  * group_size == 128 (others: WQ_ERR_UNSUPPORTED, [P4] sec. 7.2: the group must
  * divide the kernel tile); Y bf16 [M, N]; fp32 accumulation.
  * M <= 16 runs a decode kernel (every weight byte streamed once from HBM,
- * the work split evenly over all SMs): M <= 2 on the CUDA cores while the
- * prepared X (two int8 limbs per element) fits in shared memory, i.e.
- * K <= 76800 at M = 1 and K <= 37888 at M = 2, else on the tensor cores;
+ * the work split evenly over all SMs) on the CUDA cores at M <= 2 (and at
+ * M <= 4 when K <= 8192 and N * K <= 2^26) while the prepared X (two int8
+ * limbs per element) fits in shared memory -- K <= 75776 at M = 1, 37888 at
+ * M = 2, 24576 at M = 3, 18432 at M = 4 -- and on the tensor cores otherwise;
  * larger M runs the tensor-core GEMM.
  * Requires K % 128 == 0 and N % 8 == 0.
  *

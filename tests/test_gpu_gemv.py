@@ -113,16 +113,16 @@ def test_workspace_reused_and_left_zeroed():
 
 
 def test_workspace_shared_by_both_decode_kernels():
-    """One workspace, sized for the largest request, serves the CUDA-core
-    kernel (M <= 2) and the tensor-core kernel (M = 3..16) alternately."""
+    """One workspace serves the CUDA-core kernel (M <= 4) and the tensor-core
+    kernel (M = 5..16) alternately."""
     N, K = 4096, 4096
     W = make_weight(N, K, 0.02, seed=5)
     (codes, scales, zeros), _ = quantized(W, False)
-    Xs = {M: make_activation(M, K, seed=M).cuda() for M in (1, 2, 4, 16)}
+    Xs = {M: make_activation(M, K, seed=M).cuda() for M in (1, 2, 4, 8, 16)}
     ref = {M: wq.gemm_w4a16(X, codes, scales, zeros, 128, False) for M, X in Xs.items()}
     nbytes = max(wq.lib().wq_w4a16_workspace_bytes(M, N, K) for M in Xs)
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
-    for M in (1, 4, 2, 16, 1, 4):
+    for M in (1, 8, 2, 16, 1, 4, 8):
         Y = wq.gemm_w4a16(Xs[M], codes, scales, zeros, 128, False, ws=ws)
         assert torch.equal(Y, ref[M]), M
     assert int(ws[: 4 * (N // 128)].count_nonzero()) == 0
