@@ -62,10 +62,16 @@ def _declare(L):
     L.oracle_gemm_w8a8_acc.argtypes = [_P, _P, _I64, _I64, _I64, _I64, _I64, _I64,
                                        _I64, _P]
     L.oracle_w8a8_rescale.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P]
+    L.oracle_channel_absmax.argtypes = [_P, _INT, _I64, _I64, _P]
+    L.oracle_smooth_scales.argtypes = [_P, _P, _I64, ctypes.c_double, _P]
+    L.oracle_quantize_int8_rows_smoothed.argtypes = [_P, _INT, _I64, _I64, _P, _P, _P]
+    L.oracle_quant_act_i8_smoothed.argtypes = [_P, _INT, _I64, _I64, _P, _P, _P]
     for name in ("oracle_quantize_int4", "oracle_quantize_int8_rows",
                  "oracle_quant_act_i8", "oracle_dequant_int4",
                  "oracle_dequant_int8_rows", "oracle_gemm_w4a16",
-                 "oracle_gemm_w8a8_acc", "oracle_w8a8_rescale"):
+                 "oracle_gemm_w8a8_acc", "oracle_w8a8_rescale",
+                 "oracle_channel_absmax", "oracle_smooth_scales",
+                 "oracle_quantize_int8_rows_smoothed", "oracle_quant_act_i8_smoothed"):
         getattr(L, name).restype = _INT
 
 
@@ -158,6 +164,46 @@ def quant_act_i8(X, dtype_tag=None):
     s = np.zeros((M,), np.float32)
     st = lib().oracle_quant_act_i8(_ptr(X), tag, M, K, _ptr(q), _ptr(s))
     return q, s, st
+
+
+def channel_absmax(A, dtype_tag=None):
+    """SmoothQuant statistic: max_r |A[r, k]| per column.  Returns (f32 [K], status)."""
+    A, tag = _tag_and_bits(A, dtype_tag)
+    R, K = A.shape
+    out = np.zeros((K,), np.float32)
+    st = lib().oracle_channel_absmax(_ptr(A), tag, R, K, _ptr(out))
+    return out, st
+
+
+def smooth_scales(act_absmax, w_absmax, alpha=0.5):
+    """SmoothQuant migration factors s [K] (f32).  Returns (s, status)."""
+    a = _c(act_absmax, np.float32)
+    w = _c(w_absmax, np.float32)
+    s = np.zeros(a.shape, np.float32)
+    st = lib().oracle_smooth_scales(_ptr(a), _ptr(w), a.shape[0], float(alpha), _ptr(s))
+    return s, st
+
+
+def quantize_int8_rows_smoothed(W, s, dtype_tag=None):
+    """Per-channel INT8 of W diag(s).  Returns (q int8 [N, K], scales f32 [N], status)."""
+    W, tag = _tag_and_bits(W, dtype_tag)
+    N, K = W.shape
+    s = _c(s, np.float32)
+    q = np.zeros((N, K), np.int8)
+    sc = np.zeros((N,), np.float32)
+    st = lib().oracle_quantize_int8_rows_smoothed(_ptr(W), tag, N, K, _ptr(s), _ptr(q), _ptr(sc))
+    return q, sc, st
+
+
+def quant_act_i8_smoothed(X, s, dtype_tag=None):
+    """Per-token INT8 of X diag(s)^-1.  Returns (q int8 [M, K], scales f32 [M], status)."""
+    X, tag = _tag_and_bits(X, dtype_tag)
+    M, K = X.shape
+    s = _c(s, np.float32)
+    q = np.zeros((M, K), np.int8)
+    sc = np.zeros((M,), np.float32)
+    st = lib().oracle_quant_act_i8_smoothed(_ptr(X), tag, M, K, _ptr(s), _ptr(q), _ptr(sc))
+    return q, sc, st
 
 
 def dequant_int4(codes, scales, zeros, K, group_size=128, sym=True):

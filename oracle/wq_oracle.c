@@ -14,6 +14,7 @@
 #include "wq_oracle.h"
 
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 /* ------------------------------------------------------------------------- */
@@ -433,4 +434,77 @@ int oracle_w8a8_rescale(const int32_t *acc, const float *sx, const float *sw,
       Y[(m - m0) * W + (n - n0)] = (double)acc[(m - m0) * W + (n - n0)] *
                                    (double)sx[m] * (double)sw[n];
   return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* SmoothQuant smoothing                                                      */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * [P4] sec. 4.2 moves quantization difficulty from the activations to the
+ * weights with an exact rewrite of the product, Y = (X diag(s)^-1)(diag(s) W)
+ * in the page's [in, out] weight convention.  The statistics are per input
+ * channel j: the largest |X_j| seen on calibration tokens (act_scales) and
+ * the largest |W_j| over the output channels (w_scales, clamped to >= 1e-5);
+ * the migration factor is s_j = act_j^alpha / w_j^(1 - alpha), clamped to
+ * >= 1e-5, with alpha = 0.5 the page's recommended split.
+ */
+int oracle_channel_absmax(const void *A, int dtype, int64_t R, int64_t K,
+                          float *out) {
+  if (R < 0 || K <= 0) return ORACLE_ERR_ARG;
+  int status = ORACLE_OK;
+  for (int64_t k = 0; k < K; ++k) out[k] = 0.0f;
+  for (int64_t r = 0; r < R; ++r) {
+    for (int64_t k = 0; k < K; ++k) {
+      float x = load_elem(A, dtype, r * K + k);
+      if (!isfinite(x)) {
+        status = ORACLE_ERR_NONFINITE;
+        continue;
+      }
+      if (fabsf(x) > out[k]) out[k] = fabsf(x);
+    }
+  }
+  return status;
+}
+
+int oracle_smooth_scales(const float *act, const float *w, int64_t K,
+                         double alpha, float *s) {
+  if (K <= 0 || !(alpha >= 0.0 && alpha <= 1.0)) return ORACLE_ERR_ARG;
+  for (int64_t k = 0; k < K; ++k) {
+    const float wc = w[k] < 1e-5f ? 1e-5f : w[k];      /* w_scales.clamp(min=1e-5) */
+    double v = pow((double)act[k], alpha) / pow((double)wc, 1.0 - alpha);
+    if (v < 1e-5) v = 1e-5;                            /* s.clamp(min=1e-5) */
+    s[k] = (float)v;
+  }
+  return ORACLE_OK;
+}
+
+/* diag(s) W: weight column j (input channel j) multiplied by s_j, one binary32
+ * product per element, then the per-channel INT8 quantizer. */
+int oracle_quantize_int8_rows_smoothed(const void *W, int w_dtype, int64_t N,
+                                       int64_t K, const float *s, int8_t *q,
+                                       float *scales) {
+  if (N < 0 || K <= 0) return ORACLE_ERR_ARG;
+  float *ws = (float *)malloc((size_t)(N > 0 ? N : 1) * (size_t)K * sizeof(float));
+  if (!ws) return ORACLE_ERR_ARG;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) ws[n * K + k] = load_elem(W, w_dtype, n * K + k) * s[k];
+  const int st = oracle_quantize_int8_rows(ws, ORACLE_F32, N, K, q, scales);
+  free(ws);
+  return st;
+}
+
+/* X diag(s)^-1: activation column j divided by s_j, one binary32 division per
+ * element, then the per-token INT8 quantizer. */
+int oracle_quant_act_i8_smoothed(const void *X, int x_dtype, int64_t M,
+                                 int64_t K, const float *s, int8_t *q,
+                                 float *scales) {
+  if (M < 0 || K <= 0) return ORACLE_ERR_ARG;
+  float *xs = (float *)malloc((size_t)(M > 0 ? M : 1) * (size_t)K * sizeof(float));
+  if (!xs) return ORACLE_ERR_ARG;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k) xs[m * K + k] = load_elem(X, x_dtype, m * K + k) / s[k];
+  const int st = oracle_quant_act_i8(xs, ORACLE_F32, M, K, q, scales);
+  free(xs);
+  return st;
 }

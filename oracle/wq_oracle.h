@@ -19,7 +19,7 @@
  *        (per-group granularity), sec. 4 (metadata share)
  *   [P4] "27届大模型面试准备（十九）：模型量化全攻略" sec. 2.1 (affine quantization,
  *        min-max scale), 2.2 (per-group g=128, 4.25-bit), 3 (per-tensor worked
- *        example), 6 (per-token absmax quantizer)
+ *        example), 4.2 (SmoothQuant smoothing), 6 (per-token absmax quantizer)
  *
  * Status codes returned by the oracle functions.
  */
@@ -87,6 +87,24 @@ int oracle_gemm_w4a16(const uint16_t *X, int64_t M, int64_t K,
 int oracle_gemm_w8a8_acc(const int8_t *qx, const int8_t *qw, int64_t M,
                          int64_t N, int64_t K, int64_t m0, int64_t m1,
                          int64_t n0, int64_t n1, int32_t *acc);
+
+/* SmoothQuant smoothing ([P4] sec. 4.2).
+ * Per-column maximum |A[r, k]| over the R rows of A [R, K]: act_scales when A
+ * is a calibration activation X [tokens, in], w_scales when A is W [out, in]. */
+int oracle_channel_absmax(const void *A, int dtype, int64_t R, int64_t K,
+                          float *out);
+/* s[k] = max(act[k]^alpha / max(w[k], 1e-5)^(1 - alpha), 1e-5), in binary64,
+ * rounded once to binary32; 0 <= alpha <= 1. */
+int oracle_smooth_scales(const float *act, const float *w, int64_t K,
+                         double alpha, float *s);
+/* Per-channel INT8 (as oracle_quantize_int8_rows) of W'[n, k] = W[n, k] * s[k]. */
+int oracle_quantize_int8_rows_smoothed(const void *W, int w_dtype, int64_t N,
+                                       int64_t K, const float *s, int8_t *q,
+                                       float *scales);
+/* Per-token INT8 (as oracle_quant_act_i8) of X'[m, k] = X[m, k] / s[k]. */
+int oracle_quant_act_i8_smoothed(const void *X, int x_dtype, int64_t M,
+                                 int64_t K, const float *s, int8_t *q,
+                                 float *scales);
 
 /* W8A8 rescale in fp64: Y = acc * sx[m] * sw[n] over the same window. */
 int oracle_w8a8_rescale(const int32_t *acc, const float *sx, const float *sw,
