@@ -431,7 +431,24 @@ def secondary(wq, dev, args):
     out["w8a8_us"] = round(t * 1e3, 1)
     out["w8a8_frac_int8_peak"] = round(ops / (t * 1e-3) / 1e12 / int8_peak, 3)
     out["int8_peak_tops"] = int8_peak
-    del qw, sw, X8, Y8, ws8
+
+    # SmoothQuant (alpha = 0.5) in front of the same W8A8 product: statistics,
+    # factors and the smoothed weight are offline; the timed call quantizes X/s
+    # per token and runs the int8 GEMM.  The accuracy of both variants is taken
+    # against the fp64 product of the same bf16 inputs on the first 256 rows.
+    W8 = wl8.weight(0).to(dev)
+    s8 = wq.smooth_scales(wq.channel_absmax(X8), wq.channel_absmax(W8), 0.5)
+    qws, sws = wq.quantize_i8_smooth(W8, s8)
+    t = time_flushed(lambda: wq.wq_gemm_w8a8_smooth(X8, qws, sws, s8, Y8, ws8), flush)
+    out["w8a8_smooth_tops"] = round(ops / (t * 1e-3) / 1e12, 1)
+    out["w8a8_smooth_us"] = round(t * 1e3, 1)
+    ref = X8[:256].double().cpu().numpy() @ W8.double().cpu().numpy().T
+    y_plain = wq.gemm_w8a8(X8[:256].contiguous(), qw, sw).double().cpu().numpy()
+    y_smooth = wq.gemm_w8a8_smooth(X8[:256].contiguous(), qws, sws, s8).double().cpu().numpy()
+    nrm = np.linalg.norm(ref)
+    out["w8a8_rel_err_plain"] = float(f"{np.linalg.norm(y_plain - ref) / nrm:.3e}")
+    out["w8a8_rel_err_smooth"] = float(f"{np.linalg.norm(y_smooth - ref) / nrm:.3e}")
+    del qw, sw, X8, Y8, ws8, W8, s8, qws, sws
     torch.cuda.empty_cache()
     return out
 

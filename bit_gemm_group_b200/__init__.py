@@ -39,6 +39,8 @@ EXPORTED = (
     "wq_w8a8_workspace_bytes", "wq_gemm_w8a8", "wq_get_device_status",
     "wq_status_str", "wq_last_cuda_error", "wq_selftest_wait_timeout",
     "wq_gemm_w4a16_noalloc",
+    "wq_channel_absmax", "wq_smooth_scales", "wq_quantize_i8_smooth", "wq_quant_act_i8_smooth",
+    "wq_gemm_w8a8_smooth",
 )
 
 
@@ -99,8 +101,15 @@ def _declare(L):
     L.wq_selftest_wait_timeout.restype = _INT
     L.wq_last_cuda_error.argtypes = []
     L.wq_last_cuda_error.restype = ctypes.c_char_p
+    L.wq_channel_absmax.argtypes = [_P, _INT, _I64, _I64, _P, _P]
+    L.wq_smooth_scales.argtypes = [_P, _P, _I64, ctypes.c_float, _P, _P]
+    L.wq_quantize_i8_smooth.argtypes = [_P, _INT, _I64, _I64, _P, _P, _P, _P]
+    L.wq_quant_act_i8_smooth.argtypes = [_P, _I64, _I64, _P, _P, _P, _P]
+    L.wq_gemm_w8a8_smooth.argtypes = [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _SZ, _P, _P]
     for name in ("wq_quantize_pack", "wq_dequant", "wq_gemm_w4a16", "wq_quant_act_i8",
-                 "wq_gemm_w8a8", "wq_get_device_status"):
+                 "wq_gemm_w8a8", "wq_get_device_status", "wq_channel_absmax",
+                 "wq_smooth_scales", "wq_quantize_i8_smooth", "wq_quant_act_i8_smooth",
+                 "wq_gemm_w8a8_smooth"):
         getattr(L, name).restype = _INT
 
 
@@ -194,6 +203,42 @@ def wq_gemm_w8a8(X, Wq, w_scales, Y, ws, acc_out=None, stream=None):
     _check(st, "wq_gemm_w8a8")
 
 
+def wq_channel_absmax(A, out, stream=None):
+    R, K = A.shape
+    st = lib().wq_channel_absmax(_ptr(A), _DTYPE_TAG.get(A.dtype, -1), R, K, _ptr(out),
+                                 _stream(stream))
+    _check(st, "wq_channel_absmax")
+
+
+def wq_smooth_scales(act_absmax, w_absmax, alpha, s, stream=None):
+    st = lib().wq_smooth_scales(_ptr(act_absmax), _ptr(w_absmax), act_absmax.numel(),
+                                float(alpha), _ptr(s), _stream(stream))
+    _check(st, "wq_smooth_scales")
+
+
+def wq_quantize_i8_smooth(W, s, q, scales, stream=None):
+    N, K = W.shape
+    st = lib().wq_quantize_i8_smooth(_ptr(W), _DTYPE_TAG.get(W.dtype, -1), N, K, _ptr(s),
+                                     _ptr(q), _ptr(scales), _stream(stream))
+    _check(st, "wq_quantize_i8_smooth")
+
+
+def wq_quant_act_i8_smooth(X, s, q, sx, stream=None):
+    M, K = X.shape
+    st = lib().wq_quant_act_i8_smooth(_ptr(X), M, K, _ptr(s), _ptr(q), _ptr(sx),
+                                      _stream(stream))
+    _check(st, "wq_quant_act_i8_smooth")
+
+
+def wq_gemm_w8a8_smooth(X, Wq, w_scales, s, Y, ws, acc_out=None, stream=None):
+    M, K = X.shape
+    N = Wq.shape[0]
+    st = lib().wq_gemm_w8a8_smooth(_ptr(X), M, K, _ptr(Wq), _ptr(w_scales), _ptr(s), N, _ptr(Y),
+                                   _ptr(ws), ws.numel() * ws.element_size(), _ptr(acc_out),
+                                   _stream(stream))
+    _check(st, "wq_gemm_w8a8_smooth")
+
+
 def wq_get_device_status(reset=True, stream=None):
     """Synchronize the stream and return the first kernel-detected error code."""
     return int(lib().wq_get_device_status(_stream(stream), int(bool(reset))))
@@ -273,4 +318,45 @@ def gemm_w8a8(X, Wq, w_scales, want_acc=False):
                      device=X.device)
     acc = torch.empty((M, N), dtype=torch.int32, device=X.device) if want_acc else None
     wq_gemm_w8a8(X, Wq, w_scales, Y, ws, acc)
+    return (Y, acc) if want_acc else Y
+
+
+# ------------------------------------------------------ SmoothQuant helpers
+
+def channel_absmax(A):
+    out = torch.empty((A.shape[1],), dtype=torch.float32, device=A.device)
+    wq_channel_absmax(A, out)
+    return out
+
+
+def smooth_scales(act_absmax, w_absmax, alpha=0.5):
+    s = torch.empty_like(act_absmax, dtype=torch.float32)
+    wq_smooth_scales(act_absmax, w_absmax, alpha, s)
+    return s
+
+
+def quantize_i8_smooth(W, s):
+    N, K = W.shape
+    q = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    sc = torch.empty((N,), dtype=torch.float32, device=W.device)
+    wq_quantize_i8_smooth(W, s, q, sc)
+    return q, sc
+
+
+def quant_act_i8_smooth(X, s):
+    M, K = X.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    sx = torch.empty((M,), dtype=torch.float32, device=X.device)
+    wq_quant_act_i8_smooth(X, s, q, sx)
+    return q, sx
+
+
+def gemm_w8a8_smooth(X, Wq, w_scales, s, want_acc=False):
+    M, K = X.shape
+    N = Wq.shape[0]
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    ws = torch.empty((max(1, wq_w8a8_workspace_bytes(M, K)),), dtype=torch.uint8,
+                     device=X.device)
+    acc = torch.empty((M, N), dtype=torch.int32, device=X.device) if want_acc else None
+    wq_gemm_w8a8_smooth(X, Wq, w_scales, s, Y, ws, acc)
     return (Y, acc) if want_acc else Y

@@ -199,12 +199,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 namespace wq_host {
 
 int launch_gemm_w8a8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
-                     int64_t N, void* Y, void* ws, void* acc_out, cudaStream_t s) {
+                     const float* smooth, int64_t N, void* Y, void* ws, void* acc_out,
+                     cudaStream_t s) {
   using namespace wq::w8a8;
   int8_t* qx = static_cast<int8_t*>(ws);
   float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
                                        ((size_t(M) * size_t(K) + 255) & ~size_t(255)));
-  int st = launch_quantize_rows_i8(X, WQ_BF16, M, K, true, qx, sx, s);
+  int st = launch_quantize_rows_i8(X, WQ_BF16, M, K, true, smooth, qx, sx, s);
   if (st != WQ_OK) return st;
 
   CUtensorMap ta, tb;

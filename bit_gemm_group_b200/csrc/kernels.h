@@ -9,8 +9,14 @@ namespace wq_host {
 
 int launch_quantize_int4(const void* W, int w_dtype, int64_t N, int64_t K, int group_size,
                          int sym, void* codes, void* scales, void* zeros, cudaStream_t s);
+// smooth (nullable): SmoothQuant factors s [K]; activations are divided by
+// them, weights multiplied, before quantization.
 int launch_quantize_rows_i8(const void* W, int w_dtype, int64_t N, int64_t K, bool activation,
-                            void* q, void* scales, cudaStream_t s);
+                            const float* smooth, void* q, void* scales, cudaStream_t s);
+int launch_channel_absmax(const void* A, int a_dtype, int64_t R, int64_t K, float* out,
+                          cudaStream_t s);
+int launch_smooth_scales(const float* act, const float* w, int64_t K, float alpha, float* out,
+                         cudaStream_t s);
 int launch_dequant_int4(const void* codes, const void* scales, const void* zeros, int64_t N,
                         int64_t K, int group_size, int sym, void* out, int out_dtype,
                         cudaStream_t s);
@@ -42,6 +48,7 @@ int launch_gemm_w4a16(const void* X, int64_t M, int64_t K, const void* codes,
                       cudaStream_t s);
 
 int launch_gemm_w8a8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
-                     int64_t N, void* Y, void* ws, void* acc_out, cudaStream_t s);
+                     const float* smooth, int64_t N, void* Y, void* ws, void* acc_out,
+                     cudaStream_t s);
 
 }  // namespace wq_host

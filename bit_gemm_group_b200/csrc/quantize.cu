@@ -151,10 +151,24 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(
 // One 256-thread block per row: pass 1 reduces amax with 16-byte loads, pass 2
 // re-reads the row (L1/L2 resident: a row is at most a few tens of KB) and
 // writes int8 codes 8 at a time.
+// Element e of an 8-vector at column k after the optional SmoothQuant
+// migration ("27届大模型面试准备（十九）…" sec. 4.2): activations are divided by
+// s[k] (X diag(s)^-1), weights multiplied (W diag(s)); one IEEE operation.
+template <bool ACT>
+__device__ __forceinline__ void smooth8(float (&x)[8], const float* __restrict__ smooth,
+                                        int64_t k) {
+  if (smooth == nullptr) return;
+  const float4 a = *reinterpret_cast<const float4*>(smooth + k);
+  const float4 b = *reinterpret_cast<const float4*>(smooth + k + 4);
+  const float sv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) x[e] = ACT ? div_rn(x[e], sv[e]) : __fmul_rn(x[e], sv[e]);
+}
+
 template <typename T, bool ACT>
 __global__ void __launch_bounds__(256) quantize_rows_i8_kernel(
-    const T* __restrict__ X, int64_t rows, int64_t K, int8_t* __restrict__ q,
-    float* __restrict__ scales, int* status) {
+    const T* __restrict__ X, int64_t rows, int64_t K, const float* __restrict__ smooth,
+    int8_t* __restrict__ q, float* __restrict__ scales, int* status) {
   constexpr int EV = 8;  // elements per vector step
   __shared__ float red[8];
   __shared__ int bad_any;
@@ -165,11 +179,14 @@ __global__ void __launch_bounds__(256) quantize_rows_i8_kernel(
     for (int64_t k = int64_t(threadIdx.x) * EV; k < K; k += int64_t(blockDim.x) * EV) {
       Elems<T, EV> v;
       v.load(row + k);
+      float x[EV];
+#pragma unroll
+      for (int e = 0; e < EV; ++e) x[e] = to_f32<T>(v.u.e[e]);
+      smooth8<ACT>(x, smooth, k);
 #pragma unroll
       for (int e = 0; e < EV; ++e) {
-        const float x = to_f32<T>(v.u.e[e]);
-        finite &= isfinite(x);
-        amax = fmaxf(amax, fabsf(x));
+        finite &= isfinite(x[e]);
+        amax = fmaxf(amax, fabsf(x[e]));
       }
     }
     amax = warp_max(amax);
@@ -200,6 +217,10 @@ __global__ void __launch_bounds__(256) quantize_rows_i8_kernel(
     for (int64_t k = int64_t(threadIdx.x) * EV; k < K; k += int64_t(blockDim.x) * EV) {
       Elems<T, EV> v;
       v.load(row + k);
+      float x[EV];
+#pragma unroll
+      for (int e = 0; e < EV; ++e) x[e] = to_f32<T>(v.u.e[e]);
+      smooth8<ACT>(x, smooth, k);
       union {
         uint2 v2;
         int8_t b[EV];
@@ -208,7 +229,7 @@ __global__ void __launch_bounds__(256) quantize_rows_i8_kernel(
       for (int e = 0; e < EV; ++e) {
         int qi = 0;
         if (!degenerate) {
-          float rr = round_even(div_rn(to_f32<T>(v.u.e[e]), s));
+          float rr = round_even(div_rn(x[e], s));
           rr = fmaxf(-200.f, fminf(200.f, rr));
           qi = min(max(int(rr), lo), 127);
         }
@@ -218,6 +239,56 @@ __global__ void __launch_bounds__(256) quantize_rows_i8_kernel(
     }
     __syncthreads();  // red[] is reused by the next row
   }
+}
+
+// ---------------------------------------------------------------------------
+// SmoothQuant statistics ("27届大模型面试准备（十九）…" sec. 4.2)
+// ---------------------------------------------------------------------------
+// out[k] = max_r |A[r, k]| over the rows of A [R, K]: act_scales for a
+// calibration activation, w_scales for a weight [out, in].  Each thread keeps
+// eight adjacent columns (one 16- or 32-byte load per row) over a strip of
+// rows and merges with atomicMax on the bit patterns (non-negative floats
+// order like their bits), so the result does not depend on the order.
+// Non-finite elements are skipped and reported, as in the oracle.
+template <typename T>
+__global__ void __launch_bounds__(256) channel_absmax_kernel(const T* __restrict__ A, int64_t R,
+                                                             int64_t K,
+                                                             unsigned* __restrict__ out,
+                                                             int* status) {
+  const int64_t col = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  if (col >= K) return;
+  float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  bool bad = false;
+  for (int64_t r = blockIdx.y; r < R; r += gridDim.y) {
+    Elems<T, 8> v;
+    v.load(A + r * K + col);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float x = to_f32<T>(v.u.e[e]);
+      if (isfinite(x)) {
+        m[e] = fmaxf(m[e], fabsf(x));
+      } else {
+        bad = true;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) atomicMax(out + col + e, __float_as_uint(m[e]));
+  if (bad) record_error(status, WQ_ERR_NONFINITE);
+}
+
+// s[k] = max(act[k]^alpha / max(w[k], 1e-5)^(1 - alpha), 1e-5), evaluated in
+// binary64 and rounded once to binary32 (the page's smooth_ln_linear clamps).
+__global__ void __launch_bounds__(256) smooth_scales_kernel(const float* __restrict__ act,
+                                                            const float* __restrict__ w,
+                                                            int64_t K, double alpha,
+                                                            float* __restrict__ s) {
+  const int64_t k = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+  const float wc = fmaxf(w[k], 1e-5f);
+  double v = pow(double(act[k]), alpha) / pow(double(wc), 1.0 - alpha);
+  if (v < 1e-5) v = 1e-5;
+  s[k] = __double2float_rn(v);
 }
 
 // ---------------------------------------------------------------------------
@@ -361,7 +432,7 @@ int launch_quantize_int4(const void* W, int w_dtype, int64_t N, int64_t K, int g
 }
 
 int launch_quantize_rows_i8(const void* W, int w_dtype, int64_t N, int64_t K, bool activation,
-                            void* q, void* scales, cudaStream_t s) {
+                            const float* smooth, void* q, void* scales, cudaStream_t s) {
   const int grid = int(N < int64_t(sm_count()) * 16 ? N : int64_t(sm_count()) * 16);
   int* st = status_ptr();
   auto* qo = static_cast<int8_t*>(q);
@@ -370,10 +441,10 @@ int launch_quantize_rows_i8(const void* W, int w_dtype, int64_t N, int64_t K, bo
   do {                                                                                       \
     if (activation)                                                                          \
       wq::quantize_rows_i8_kernel<T, true><<<grid, 256, 0, s>>>(static_cast<const T*>(W), N, \
-                                                                K, qo, so, st);              \
+                                                                K, smooth, qo, so, st);      \
     else                                                                                     \
       wq::quantize_rows_i8_kernel<T, false><<<grid, 256, 0, s>>>(static_cast<const T*>(W),   \
-                                                                 N, K, qo, so, st);          \
+                                                                 N, K, smooth, qo, so, st);  \
   } while (0)
   switch (w_dtype) {
     case WQ_F32: WQ_ROWS(float); break;
@@ -383,6 +454,41 @@ int launch_quantize_rows_i8(const void* W, int w_dtype, int64_t N, int64_t K, bo
   }
 #undef WQ_ROWS
   WQ_LAUNCH_CHECK("quantize_rows_i8_kernel");
+  return WQ_OK;
+}
+
+int launch_channel_absmax(const void* A, int a_dtype, int64_t R, int64_t K, float* out,
+                          cudaStream_t s) {
+  WQ_CUDA_CHECK(cudaMemsetAsync(out, 0, size_t(K) * 4, s));
+  if (R == 0) return WQ_OK;
+  const int64_t groups = K / 8;  // 8 columns per thread
+  const int gx = int((groups + 255) / 256);
+  const int64_t want = int64_t(sm_count()) * 8;
+  const int gy = int(R < want / gx + 1 ? R : want / gx + 1);
+  const dim3 grid(unsigned(gx), unsigned(gy > 65535 ? 65535 : gy));
+  auto* o = reinterpret_cast<unsigned*>(out);
+  int* st = status_ptr();
+  switch (a_dtype) {
+    case WQ_F32:
+      wq::channel_absmax_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(A), R, K, o, st);
+      break;
+    case WQ_BF16:
+      wq::channel_absmax_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(A), R, K, o, st);
+      break;
+    case WQ_F16:
+      wq::channel_absmax_kernel<__half><<<grid, 256, 0, s>>>(static_cast<const __half*>(A), R, K, o, st);
+      break;
+    default: return WQ_ERR_ARG;
+  }
+  WQ_LAUNCH_CHECK("channel_absmax_kernel");
+  return WQ_OK;
+}
+
+int launch_smooth_scales(const float* act, const float* w, int64_t K, float alpha, float* out,
+                         cudaStream_t s) {
+  wq::smooth_scales_kernel<<<grid_for(K, 256), 256, 0, s>>>(act, w, K, double(alpha), out);
+  WQ_LAUNCH_CHECK("smooth_scales_kernel");
   return WQ_OK;
 }
 

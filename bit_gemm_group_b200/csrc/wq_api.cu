@@ -119,7 +119,7 @@ int wq_quantize_pack(const void* W, int w_dtype, int64_t N, int64_t K, int group
   if (bits == 4)
     return wq_host::launch_quantize_int4(W, w_dtype, N, K, group_size, sym, codes, scales, zeros,
                                          as_stream(stream));
-  return wq_host::launch_quantize_rows_i8(W, w_dtype, N, K, false, codes, scales,
+  return wq_host::launch_quantize_rows_i8(W, w_dtype, N, K, false, nullptr, codes, scales,
                                           as_stream(stream));
 }
 
@@ -190,7 +190,7 @@ int wq_quant_act_i8(const void* X, int64_t M, int64_t K, void* q, void* s, void*
   if (!aligned16(X) || !aligned16(q) || !aligned16(s)) return WQ_ERR_ALIGN;
   int st = wq_host::ensure_device();
   if (st != WQ_OK) return st;
-  return wq_host::launch_quantize_rows_i8(X, WQ_BF16, M, K, true, q, s, as_stream(stream));
+  return wq_host::launch_quantize_rows_i8(X, WQ_BF16, M, K, true, nullptr, q, s, as_stream(stream));
 }
 
 size_t wq_w8a8_workspace_bytes(int64_t M, int64_t K) {
@@ -215,7 +215,89 @@ int wq_gemm_w8a8(const void* X, int64_t M, int64_t K, const void* Wq, const void
     return WQ_ERR_ALIGN;
   int st = wq_host::ensure_device();
   if (st != WQ_OK) return st;
-  return wq_host::launch_gemm_w8a8(X, M, K, Wq, w_scales, N, Y, ws, acc_out, as_stream(stream));
+  return wq_host::launch_gemm_w8a8(X, M, K, Wq, w_scales, nullptr, N, Y, ws, acc_out,
+                                   as_stream(stream));
+}
+
+// ------------------------------------------------------------- SmoothQuant
+
+int wq_channel_absmax(const void* A, int a_dtype, int64_t R, int64_t K, void* out,
+                      void* stream) {
+  if (R < 0 || K < 0) return WQ_ERR_ARG;
+  if (a_dtype != WQ_F32 && a_dtype != WQ_BF16 && a_dtype != WQ_F16) return WQ_ERR_ARG;
+  if ((K % 8) != 0) return WQ_ERR_ALIGN;
+  if (K == 0) return WQ_OK;
+  if (!out || (R > 0 && !A)) return WQ_ERR_ARG;
+  if ((A && !aligned16(A)) || !aligned16(out)) return WQ_ERR_ALIGN;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  return wq_host::launch_channel_absmax(A, a_dtype, R, K, static_cast<float*>(out),
+                                        as_stream(stream));
+}
+
+int wq_smooth_scales(const void* act_absmax, const void* w_absmax, int64_t K, float alpha,
+                     void* s, void* stream) {
+  if (K < 0) return WQ_ERR_ARG;
+  if (!(alpha >= 0.f && alpha <= 1.f)) return WQ_ERR_ARG;
+  if (K == 0) return WQ_OK;
+  if (!act_absmax || !w_absmax || !s) return WQ_ERR_ARG;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  return wq_host::launch_smooth_scales(static_cast<const float*>(act_absmax),
+                                       static_cast<const float*>(w_absmax), K, alpha,
+                                       static_cast<float*>(s), as_stream(stream));
+}
+
+int wq_quantize_i8_smooth(const void* W, int w_dtype, int64_t N, int64_t K, const void* smooth,
+                          void* q, void* scales, void* stream) {
+  if (N < 0 || K < 0) return WQ_ERR_ARG;
+  if (w_dtype != WQ_F32 && w_dtype != WQ_BF16 && w_dtype != WQ_F16) return WQ_ERR_ARG;
+  if ((K % 16) != 0) return WQ_ERR_ALIGN;
+  if (N == 0 || K == 0) return WQ_OK;
+  if (!W || !smooth || !q || !scales) return WQ_ERR_ARG;
+  if (!aligned16(W) || !aligned16(smooth) || !aligned16(q) || !aligned16(scales))
+    return WQ_ERR_ALIGN;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  return wq_host::launch_quantize_rows_i8(W, w_dtype, N, K, false,
+                                          static_cast<const float*>(smooth), q, scales,
+                                          as_stream(stream));
+}
+
+int wq_quant_act_i8_smooth(const void* X, int64_t M, int64_t K, const void* smooth, void* q,
+                           void* s, void* stream) {
+  if (M < 0 || K < 0) return WQ_ERR_ARG;
+  if ((K % 16) != 0) return WQ_ERR_ALIGN;
+  if (M == 0 || K == 0) return WQ_OK;
+  if (!X || !smooth || !q || !s) return WQ_ERR_ARG;
+  if (!aligned16(X) || !aligned16(smooth) || !aligned16(q) || !aligned16(s)) return WQ_ERR_ALIGN;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  return wq_host::launch_quantize_rows_i8(X, WQ_BF16, M, K, true,
+                                          static_cast<const float*>(smooth), q, s,
+                                          as_stream(stream));
+}
+
+int wq_gemm_w8a8_smooth(const void* X, int64_t M, int64_t K, const void* Wq,
+                        const void* w_scales, const void* smooth, int64_t N, void* Y, void* ws,
+                        size_t ws_bytes, void* acc_out, void* stream) {
+  if (!smooth) return WQ_ERR_ARG;
+  if (!aligned16(smooth)) return WQ_ERR_ALIGN;
+  if (M < 0 || K < 0 || N < 0) return WQ_ERR_ARG;
+  if ((K % 16) != 0 || (N % 16) != 0) return WQ_ERR_ALIGN;
+  if (M > (int64_t(1) << 31) / 2 || N > (int64_t(1) << 31) / 2 || K > (int64_t(1) << 24))
+    return WQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return WQ_OK;
+  if (K == 0) return WQ_ERR_ARG;
+  if (!X || !Wq || !w_scales || !Y) return WQ_ERR_ARG;
+  if (!ws || ws_bytes < wq_w8a8_workspace_bytes(M, K)) return WQ_ERR_WORKSPACE;
+  if (!aligned16(X) || !aligned16(Wq) || !aligned16(w_scales) || !aligned16(Y) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || (acc_out && !aligned16(acc_out)))
+    return WQ_ERR_ALIGN;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  return wq_host::launch_gemm_w8a8(X, M, K, Wq, w_scales, static_cast<const float*>(smooth), N,
+                                   Y, ws, acc_out, as_stream(stream));
 }
 
 int wq_get_device_status(void* stream, int reset) {

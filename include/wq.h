@@ -188,6 +188,62 @@ WQ_API int wq_gemm_w8a8(const void *X, int64_t M, int64_t K, const void *Wq,
                  size_t ws_bytes, void *acc_out, void *stream);
 
 /*
+ * SmoothQuant smoothing ([P4] sec. 4.2): Y = (X diag(s)^-1)(diag(s) W) moves
+ * quantization difficulty from activations with outlier channels to the
+ * weights, with s_j = max|X_j|^alpha / max|W_j|^(1 - alpha) per input
+ * channel j.  The five calls below compute the statistics and s, quantize the
+ * smoothed weight and activations, and run the W8A8 product on them.
+ */
+
+/*
+ * wq_channel_absmax -- out[k] = max_r |A[r, k]| over the R rows of A [R, K]
+ * (a_dtype WQ_F32 / WQ_BF16 / WQ_F16): act_scales when A is calibration
+ * activations [tokens, K], w_scales when A is a weight [N, K].  out fp32 [K].
+ * Requires K % 8 == 0.  Non-finite elements are skipped and reported as
+ * WQ_ERR_NONFINITE in the device status.
+ */
+WQ_API int wq_channel_absmax(const void *A, int a_dtype, int64_t R, int64_t K,
+                             void *out, void *stream);
+
+/*
+ * wq_smooth_scales -- s[k] = max(act[k]^alpha / max(w[k], 1e-5)^(1 - alpha),
+ * 1e-5) for fp32 [K] statistics, evaluated in binary64 and rounded to fp32
+ * (the clamps of [P4] sec. 4.2's smooth_ln_linear).  0 <= alpha <= 1; the
+ * page recommends 0.5.
+ */
+WQ_API int wq_smooth_scales(const void *act_absmax, const void *w_absmax,
+                            int64_t K, float alpha, void *s, void *stream);
+
+/*
+ * wq_quantize_i8_smooth -- per-output-channel INT8 (as wq_quantize_pack with
+ * bits = 8) of the smoothed weight W'[n, k] = W[n, k] * s[k] (one fp32 product
+ * per element; W' is never stored).  W [N, K] of w_dtype, s fp32 [K] -> q int8
+ * [N, K], scales fp32 [N].  Requires K % 16 == 0.
+ */
+WQ_API int wq_quantize_i8_smooth(const void *W, int w_dtype, int64_t N, int64_t K,
+                                 const void *s, void *q, void *scales, void *stream);
+
+/*
+ * wq_quant_act_i8_smooth -- per-token INT8 (as wq_quant_act_i8) of the
+ * smoothed activations X'[m, k] = X[m, k] / s[k] (one IEEE fp32 division per
+ * element).  X bf16 [M, K], s fp32 [K] -> q int8 [M, K], sx fp32 [M].
+ * Requires K % 16 == 0.
+ */
+WQ_API int wq_quant_act_i8_smooth(const void *X, int64_t M, int64_t K, const void *s,
+                                  void *q, void *sx, void *stream);
+
+/*
+ * wq_gemm_w8a8_smooth -- wq_gemm_w8a8 on the smoothed pair: X is quantized
+ * per token after division by s (as wq_quant_act_i8_smooth) into `ws`, then
+ * multiplied with Wq / w_scales from wq_quantize_i8_smooth with the same s.
+ * Same arguments, requirements and workspace as wq_gemm_w8a8, plus s fp32 [K].
+ */
+WQ_API int wq_gemm_w8a8_smooth(const void *X, int64_t M, int64_t K, const void *Wq,
+                               const void *w_scales, const void *s, int64_t N,
+                               void *Y, void *ws, size_t ws_bytes, void *acc_out,
+                               void *stream);
+
+/*
  * wq_get_device_status -- synchronize `stream`, then return the first error
  * any kernel recorded since the last reset (WQ_OK if none); clear it when
  * reset != 0.  Returns WQ_ERR_CUDA if the synchronization itself fails.

@@ -98,3 +98,22 @@ def test_binding_refuses_cpu_tensors(L):
 def test_oracle_builds():
     import oracle
     assert os.path.exists(oracle.build.build())
+
+
+def test_smoothquant_validation(L):
+    # host-side checks return before any device work
+    assert L.wq_channel_absmax(FAKE, 1, 8, 12, FAKE, None) == wq.WQ_ERR_ALIGN          # K % 8
+    assert L.wq_channel_absmax(FAKE, 9, 8, 16, FAKE, None) == wq.WQ_ERR_ARG            # dtype
+    assert L.wq_channel_absmax(MISALIGNED, 1, 8, 16, FAKE, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_channel_absmax(FAKE, 1, 8, 0, FAKE, None) == wq.WQ_OK
+    assert L.wq_smooth_scales(FAKE, FAKE, 16, 1.5, FAKE, None) == wq.WQ_ERR_ARG        # alpha
+    assert L.wq_smooth_scales(FAKE, FAKE, 16, -0.1, FAKE, None) == wq.WQ_ERR_ARG
+    assert L.wq_smooth_scales(None, FAKE, 16, 0.5, FAKE, None) == wq.WQ_ERR_ARG
+    assert L.wq_quantize_i8_smooth(FAKE, 1, 8, 24, FAKE, FAKE, FAKE, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_quantize_i8_smooth(FAKE, 1, 8, 32, None, FAKE, FAKE, None) == wq.WQ_ERR_ARG
+    assert L.wq_quant_act_i8_smooth(FAKE, 8, 32, None, FAKE, FAKE, None) == wq.WQ_ERR_ARG
+    assert L.wq_quant_act_i8_smooth(FAKE, 8, 40, FAKE, FAKE, FAKE, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_gemm_w8a8_smooth(FAKE, 8, 128, FAKE, FAKE, None, 16, FAKE, FAKE, 1 << 20,
+                                 None, None) == wq.WQ_ERR_ARG
+    assert L.wq_gemm_w8a8_smooth(FAKE, 8, 128, FAKE, FAKE, FAKE, 16, FAKE, FAKE, 0,
+                                 None, None) == wq.WQ_ERR_WORKSPACE
