@@ -66,12 +66,14 @@ def _declare(L):
     L.oracle_smooth_scales.argtypes = [_P, _P, _I64, ctypes.c_double, _P]
     L.oracle_quantize_int8_rows_smoothed.argtypes = [_P, _INT, _I64, _I64, _P, _P, _P]
     L.oracle_quant_act_i8_smoothed.argtypes = [_P, _INT, _I64, _I64, _P, _P, _P]
+    L.oracle_quant_kv.argtypes = [_P, _P, _INT, _I64, _I64, _I64, _P, _P, _P, _P]
     for name in ("oracle_quantize_int4", "oracle_quantize_int8_rows",
                  "oracle_quant_act_i8", "oracle_dequant_int4",
                  "oracle_dequant_int8_rows", "oracle_gemm_w4a16",
                  "oracle_gemm_w8a8_acc", "oracle_w8a8_rescale",
                  "oracle_channel_absmax", "oracle_smooth_scales",
-                 "oracle_quantize_int8_rows_smoothed", "oracle_quant_act_i8_smoothed"):
+                 "oracle_quantize_int8_rows_smoothed", "oracle_quant_act_i8_smoothed",
+                 "oracle_quant_kv"):
         getattr(L, name).restype = _INT
 
 
@@ -204,6 +206,22 @@ def quant_act_i8_smoothed(X, s, dtype_tag=None):
     sc = np.zeros((M,), np.float32)
     st = lib().oracle_quant_act_i8_smoothed(_ptr(X), tag, M, K, _ptr(s), _ptr(q), _ptr(sc))
     return q, sc, st
+
+
+def quant_kv(Kc, Vc, dtype_tag=None):
+    """KV-cache INT8 of K, V [BH, S, D]: K per channel, V per token.
+    Returns (qk int8 [BH, S, D], sk f32 [BH, D], qv int8 [BH, S, D], sv f32 [BH, S], status)."""
+    Kc, tag = _tag_and_bits(Kc, dtype_tag)
+    Vc, tag2 = _tag_and_bits(Vc, dtype_tag)
+    assert tag == tag2 and Kc.shape == Vc.shape
+    BH, S, D = Kc.shape
+    qk = np.zeros((BH, S, D), np.int8)
+    qv = np.zeros((BH, S, D), np.int8)
+    sk = np.zeros((BH, D), np.float32)
+    sv = np.zeros((BH, S), np.float32)
+    st = lib().oracle_quant_kv(_ptr(Kc), _ptr(Vc), tag, BH, S, D, _ptr(qk), _ptr(sk), _ptr(qv),
+                               _ptr(sv))
+    return qk, sk, qv, sv, st
 
 
 def dequant_int4(codes, scales, zeros, K, group_size=128, sym=True):

@@ -508,3 +508,47 @@ int oracle_quant_act_i8_smoothed(const void *X, int x_dtype, int64_t M,
   free(xs);
   return st;
 }
+
+/* ------------------------------------------------------------------------- */
+/* KV-cache INT8                                                              */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * [P4] sec. 6: K and V are quantized differently.  V is flat across channels
+ * and takes one scale per token (the page's quant_kv_per_token: scale =
+ * amax over the head dim / qmax, clamped to >= 1e-8, q = clamp(round(v /
+ * scale), -qmax - 1, qmax)).  K carries channel-wise outliers (it meets Q in a
+ * dot product and carries RoPE), so it takes one scale per channel: the same
+ * quantizer with the maximum taken over the tokens of a head instead.
+ */
+int oracle_quant_kv(const void *K, const void *V, int dtype, int64_t BH,
+                    int64_t S, int64_t D, int8_t *qk, float *sk, int8_t *qv,
+                    float *sv) {
+  if (BH < 0 || S < 0 || D <= 0) return ORACLE_ERR_ARG;
+  int status = ORACLE_OK;
+  /* V: rows of D elements, the per-token quantizer as it stands */
+  if (BH * S > 0) {
+    int st = oracle_quant_act_i8(V, dtype, BH * S, D, qv, sv);
+    if (st != ORACLE_OK) status = st;
+  }
+  /* K: for each head, column d over the S tokens */
+  for (int64_t h = 0; h < BH; ++h) {
+    for (int64_t d = 0; d < D; ++d) {
+      float amax = 0.0f;
+      for (int64_t t = 0; t < S; ++t) {
+        float x = load_elem(K, dtype, (h * S + t) * D + d);
+        if (!isfinite(x)) status = ORACLE_ERR_NONFINITE;
+        if (fabsf(x) > amax) amax = fabsf(x);
+      }
+      float s = amax / 127.0f;
+      if (s < 1e-8f) s = 1e-8f;
+      sk[h * D + d] = s;
+      for (int64_t t = 0; t < S; ++t) {
+        float r = oracle_round_half_even(load_elem(K, dtype, (h * S + t) * D + d) / s);
+        r = fmaxf(-200.0f, fminf(200.0f, r));
+        qk[(h * S + t) * D + d] = (int8_t)clamp_int((int)r, -128, 127);
+      }
+    }
+  }
+  return status;
+}

@@ -19,7 +19,8 @@
  *        (per-group granularity), sec. 4 (metadata share)
  *   [P4] "27届大模型面试准备（十九）：模型量化全攻略" sec. 2.1 (affine quantization,
  *        min-max scale), 2.2 (per-group g=128, 4.25-bit), 3 (per-tensor worked
- *        example), 4.2 (SmoothQuant smoothing), 6 (per-token absmax quantizer)
+ *        example), 4.2 (SmoothQuant smoothing), 6 (per-token absmax quantizer,
+ *        KV-cache: K per channel, V per token)
  *
  * Status codes returned by the oracle functions.
  */
@@ -105,6 +106,14 @@ int oracle_quantize_int8_rows_smoothed(const void *W, int w_dtype, int64_t N,
 int oracle_quant_act_i8_smoothed(const void *X, int x_dtype, int64_t M,
                                  int64_t K, const float *s, int8_t *q,
                                  float *scales);
+
+/* KV-cache INT8 ([P4] sec. 6).  K and V are [BH, S, D] (batch x kv-heads,
+ * tokens, head dim).  V per token: sv[bh, t] = max(max_d |V| / 127, 1e-8),
+ * qv = clamp(round(V / sv), -128, 127).  K per channel: sk[bh, d] =
+ * max(max_t |K| / 127, 1e-8) over the S tokens of that head, qk likewise. */
+int oracle_quant_kv(const void *K, const void *V, int dtype, int64_t BH,
+                    int64_t S, int64_t D, int8_t *qk, float *sk, int8_t *qv,
+                    float *sv);
 
 /* W8A8 rescale in fp64: Y = acc * sx[m] * sw[n] over the same window. */
 int oracle_w8a8_rescale(const int32_t *acc, const float *sx, const float *sw,
