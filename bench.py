@@ -450,6 +450,26 @@ def secondary(wq, dev, args):
     out["w8a8_rel_err_smooth"] = float(f"{np.linalg.norm(y_smooth - ref) / nrm:.3e}")
     del qw, sw, X8, Y8, ws8, W8, s8, qws, sws
     torch.cuda.empty_cache()
+
+    # KV-cache INT8 (K per channel, V per token), bf16 cache of 8 kv heads x 8
+    # sequences x 8192 tokens x 128 dims (2 x 134 MB, larger than L2).  The
+    # algorithmic bytes count one read of K and V, the int8 writes and the
+    # scales; K is read a second time for its channel maxima.
+    BH, S, D = 64, 8192, 128
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(6)
+    Kc = torch.randn((BH, S, D), generator=gen, device=dev).to(torch.bfloat16)
+    Vc = torch.randn((BH, S, D), generator=gen, device=dev).to(torch.bfloat16)
+    qk = torch.empty((BH, S, D), dtype=torch.int8, device=dev)
+    qv = torch.empty_like(qk)
+    sk = torch.empty((BH, D), dtype=torch.float32, device=dev)
+    sv = torch.empty((BH, S), dtype=torch.float32, device=dev)
+    t = time_flushed(lambda: wq.wq_quant_kv(Kc, Vc, qk, sk, qv, sv), flush)
+    kv_bytes = 2 * BH * S * D * (2 + 1) + BH * D * 4 + BH * S * 4
+    out["kv_quant_gbs"] = round(kv_bytes / (t * 1e-3) / 1e9, 1)
+    out["kv_quant_frac_hbm"] = round(kv_bytes / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 3)
+    del Kc, Vc, qk, qv, sk, sv
+    torch.cuda.empty_cache()
     return out
 
 

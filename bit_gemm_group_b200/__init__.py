@@ -40,7 +40,7 @@ EXPORTED = (
     "wq_status_str", "wq_last_cuda_error", "wq_selftest_wait_timeout",
     "wq_gemm_w4a16_noalloc",
     "wq_channel_absmax", "wq_smooth_scales", "wq_quantize_i8_smooth", "wq_quant_act_i8_smooth",
-    "wq_gemm_w8a8_smooth",
+    "wq_gemm_w8a8_smooth", "wq_quant_kv",
 )
 
 
@@ -106,10 +106,11 @@ def _declare(L):
     L.wq_quantize_i8_smooth.argtypes = [_P, _INT, _I64, _I64, _P, _P, _P, _P]
     L.wq_quant_act_i8_smooth.argtypes = [_P, _I64, _I64, _P, _P, _P, _P]
     L.wq_gemm_w8a8_smooth.argtypes = [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _SZ, _P, _P]
+    L.wq_quant_kv.argtypes = [_P, _P, _INT, _I64, _I64, _I64, _P, _P, _P, _P, _P]
     for name in ("wq_quantize_pack", "wq_dequant", "wq_gemm_w4a16", "wq_quant_act_i8",
                  "wq_gemm_w8a8", "wq_get_device_status", "wq_channel_absmax",
                  "wq_smooth_scales", "wq_quantize_i8_smooth", "wq_quant_act_i8_smooth",
-                 "wq_gemm_w8a8_smooth"):
+                 "wq_gemm_w8a8_smooth", "wq_quant_kv"):
         getattr(L, name).restype = _INT
 
 
@@ -239,6 +240,13 @@ def wq_gemm_w8a8_smooth(X, Wq, w_scales, s, Y, ws, acc_out=None, stream=None):
     _check(st, "wq_gemm_w8a8_smooth")
 
 
+def wq_quant_kv(K, V, qk, sk, qv, sv, stream=None):
+    BH, S, D = K.shape
+    st = lib().wq_quant_kv(_ptr(K), _ptr(V), _DTYPE_TAG.get(K.dtype, -1), BH, S, D, _ptr(qk),
+                           _ptr(sk), _ptr(qv), _ptr(sv), _stream(stream))
+    _check(st, "wq_quant_kv")
+
+
 def wq_get_device_status(reset=True, stream=None):
     """Synchronize the stream and return the first kernel-detected error code."""
     return int(lib().wq_get_device_status(_stream(stream), int(bool(reset))))
@@ -360,3 +368,14 @@ def gemm_w8a8_smooth(X, Wq, w_scales, s, want_acc=False):
     acc = torch.empty((M, N), dtype=torch.int32, device=X.device) if want_acc else None
     wq_gemm_w8a8_smooth(X, Wq, w_scales, s, Y, ws, acc)
     return (Y, acc) if want_acc else Y
+
+
+def quant_kv(K, V):
+    """KV-cache INT8 of K, V [BH, S, D]: (qk, sk [BH, D], qv, sv [BH, S])."""
+    BH, S, D = K.shape
+    qk = torch.empty((BH, S, D), dtype=torch.int8, device=K.device)
+    qv = torch.empty((BH, S, D), dtype=torch.int8, device=K.device)
+    sk = torch.empty((BH, D), dtype=torch.float32, device=K.device)
+    sv = torch.empty((BH, S), dtype=torch.float32, device=K.device)
+    wq_quant_kv(K, V, qk, sk, qv, sv)
+    return qk, sk, qv, sv

@@ -17,6 +17,8 @@ int launch_channel_absmax(const void* A, int a_dtype, int64_t R, int64_t K, floa
                           cudaStream_t s);
 int launch_smooth_scales(const float* act, const float* w, int64_t K, float alpha, float* out,
                          cudaStream_t s);
+int launch_quant_kv(const void* Kc, const void* Vc, int dtype, int64_t BH, int64_t S, int64_t D,
+                    void* qk, void* sk, void* qv, void* sv, cudaStream_t s);
 int launch_dequant_int4(const void* codes, const void* scales, const void* zeros, int64_t N,
                         int64_t K, int group_size, int sym, void* out, int out_dtype,
                         cudaStream_t s);

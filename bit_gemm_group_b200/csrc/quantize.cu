@@ -292,6 +292,139 @@ __global__ void __launch_bounds__(256) smooth_scales_kernel(const float* __restr
 }
 
 // ---------------------------------------------------------------------------
+// KV-cache INT8 ("27届大模型面试准备（十九）…" sec. 6)
+// ---------------------------------------------------------------------------
+// K [BH, S, D] per channel: amax over the S tokens of each (head, channel).
+// Block (D/8 column groups) x (256 / (D/8) token rows); CTA (strip, bh) walks
+// its strip of tokens, reduces its rows in shared memory and merges with
+// atomicMax on the fp32 bit patterns (order-free, like channel_absmax).
+template <typename T>
+__global__ void __launch_bounds__(256) kv_k_absmax_kernel(const T* __restrict__ Kc, int64_t S,
+                                                          int D, unsigned* __restrict__ amax,
+                                                          int* status) {
+  __shared__ float red[256 * 8];
+  const int cg = threadIdx.x % (D / 8), ty = threadIdx.x / (D / 8);
+  const int rows = blockDim.x / (D / 8);
+  const int64_t bh = blockIdx.y;
+  const T* base = Kc + bh * S * D + cg * 8;
+  float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  bool bad = false;
+  for (int64_t t = int64_t(blockIdx.x) * rows + ty; t < S; t += int64_t(gridDim.x) * rows) {
+    Elems<T, 8> v;
+    v.load(base + t * D);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float x = to_f32<T>(v.u.e[e]);
+      if (isfinite(x)) {
+        m[e] = fmaxf(m[e], fabsf(x));
+      } else {
+        bad = true;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[threadIdx.x * 8 + e] = m[e];
+  __syncthreads();
+  if (ty == 0) {
+    for (int r = 1; r < rows; ++r)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], red[(r * (D / 8) + cg) * 8 + e]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) atomicMax(amax + bh * D + cg * 8 + e, __float_as_uint(m[e]));
+  }
+  if (bad) record_error(status, WQ_ERR_NONFINITE);
+}
+
+// V [rows = BH S, D] per token, for head dims D = 8 LPR with LPR a power of two
+// <= 32: a row is LPR lanes of eight elements, a warp holds 32 / LPR rows, and
+// the row maximum is a shuffle reduction inside the row's lane segment (no
+// shared memory, no block barrier).  Same arithmetic as the per-token
+// quantizer: s = max(amax / 127, 1e-8), q = clamp(round(v / s), -128, 127).
+template <typename T, int LPR>
+__global__ void __launch_bounds__(256) kv_v_quant_kernel(const T* __restrict__ V, int64_t rows,
+                                                         int8_t* __restrict__ qv,
+                                                         float* __restrict__ sv, int* status) {
+  constexpr int D = 8 * LPR;
+  constexpr int RPW = 32 / LPR;  // rows per warp
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, seg = lane % LPR;
+  const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  bool bad = false;
+  for (int64_t r0 = warp * RPW; r0 < rows; r0 += nwarps * RPW) {
+    const int64_t r = r0 + sub;
+    const bool act = r < rows;
+    float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (act) {
+      Elems<T, 8> v;
+      v.load(V + r * D + seg * 8);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = to_f32<T>(v.u.e[e]);
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      bad |= !isfinite(x[e]);
+      amax = fmaxf(amax, fabsf(x[e]));
+    }
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sc = fmaxf(div_rn(amax, 127.f), 1e-8f);
+    if (act) {
+      union {
+        uint2 v2;
+        int8_t b8[8];
+      } o;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float rr = round_even(div_rn(x[e], sc));
+        rr = fmaxf(-200.f, fminf(200.f, rr));
+        o.b8[e] = int8_t(min(max(int(rr), -128), 127));
+      }
+      *reinterpret_cast<uint2*>(qv + r * D + seg * 8) = o.v2;
+      if (seg == 0) sv[r] = sc;
+    }
+  }
+  if (bad) record_error(status, WQ_ERR_NONFINITE);
+}
+
+// sk = max(amax / 127, 1e-8) in place (amax arrives as fp32 bit patterns).
+__global__ void __launch_bounds__(256) kv_k_scale_kernel(float* __restrict__ sk, int64_t n) {
+  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) sk[i] = fmaxf(div_rn(sk[i], 127.f), 1e-8f);
+}
+
+// qk = clamp(round(K / sk[bh, d]), -128, 127), eight channels per thread.
+template <typename T>
+__global__ void __launch_bounds__(256) kv_k_quant_kernel(const T* __restrict__ Kc, int64_t S,
+                                                         int D, const float* __restrict__ sk,
+                                                         int8_t* __restrict__ qk,
+                                                         int64_t n8) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t e0 = i * 8;                  // first element
+    const int64_t bh = e0 / (S * D);
+    const int d0 = int(e0 % D);
+    Elems<T, 8> v;
+    v.load(Kc + e0);
+    const float4 a = *reinterpret_cast<const float4*>(sk + bh * D + d0);
+    const float4 b = *reinterpret_cast<const float4*>(sk + bh * D + d0 + 4);
+    const float sc[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    union {
+      uint2 v2;
+      int8_t b8[8];
+    } o;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float r = round_even(div_rn(to_f32<T>(v.u.e[e]), sc[e]));
+      r = fmaxf(-200.f, fminf(200.f, r));
+      o.b8[e] = int8_t(min(max(int(r), -128), 127));
+    }
+    *reinterpret_cast<uint2*>(qk + e0) = o.v2;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Dequantization
 // ---------------------------------------------------------------------------
 // One thread expands 16 bytes of codes (32 elements) of one row.
@@ -482,6 +615,68 @@ int launch_channel_absmax(const void* A, int a_dtype, int64_t R, int64_t K, floa
     default: return WQ_ERR_ARG;
   }
   WQ_LAUNCH_CHECK("channel_absmax_kernel");
+  return WQ_OK;
+}
+
+int launch_quant_kv(const void* Kc, const void* Vc, int dtype, int64_t BH, int64_t S, int64_t D,
+                    void* qk, void* sk, void* qv, void* sv, cudaStream_t s) {
+  float* skf = static_cast<float*>(sk);
+  WQ_CUDA_CHECK(cudaMemsetAsync(skf, 0, size_t(BH) * size_t(D) * 4, s));
+  if (BH == 0 || S == 0) return WQ_OK;
+  const int groups = int(D / 8);
+  const int rows = 256 / groups;
+  const int64_t want = int64_t(sm_count()) * 8 / BH + 1;
+  const int64_t strips_need = (S + rows - 1) / rows;
+  const int strips = int(strips_need < want ? strips_need : want);
+  const dim3 ga(unsigned(strips > 65535 ? 65535 : strips), unsigned(BH));
+  const int block = groups * rows;
+  const int64_t n8 = BH * S * D / 8;
+  int* st = status_ptr();
+  auto* am = reinterpret_cast<unsigned*>(skf);
+  auto* q8 = static_cast<int8_t*>(qk);
+#define WQ_KV(T)                                                                               \
+  do {                                                                                         \
+    wq::kv_k_absmax_kernel<T><<<ga, block, 0, s>>>(static_cast<const T*>(Kc), S, int(D), am,  \
+                                                   st);                                        \
+    wq::kv_k_scale_kernel<<<grid_for(BH * D, 256), 256, 0, s>>>(skf, BH * D);                  \
+    wq::kv_k_quant_kernel<T><<<grid_for(n8, 256), 256, 0, s>>>(static_cast<const T*>(Kc), S,   \
+                                                               int(D), skf, q8, n8);           \
+  } while (0)
+  switch (dtype) {
+    case WQ_F32: WQ_KV(float); break;
+    case WQ_BF16: WQ_KV(__nv_bfloat16); break;
+    case WQ_F16: WQ_KV(__half); break;
+    default: return WQ_ERR_ARG;
+  }
+#undef WQ_KV
+  WQ_LAUNCH_CHECK("kv_k_quant_kernel");
+  // V: one scale per token row of D elements
+  const int64_t vrows = BH * S;
+  const int lpr = int(D / 8);
+  if ((lpr & (lpr - 1)) != 0)  // head dims that are not 8 x a power of two
+    return launch_quantize_rows_i8(Vc, dtype, vrows, D, true, nullptr, qv, sv, s);
+  const int64_t warps_needed = (vrows * lpr + 31) / 32;
+  const int vgrid = grid_for(warps_needed * 32, 256);
+  auto* qvo = static_cast<int8_t*>(qv);
+  auto* svo = static_cast<float*>(sv);
+#define WQ_KVV(T, L)                                                                             \
+  case L:                                                                                        \
+    wq::kv_v_quant_kernel<T, L><<<vgrid, 256, 0, s>>>(static_cast<const T*>(Vc), vrows, qvo, svo, \
+                                                      st);                                       \
+    break;
+#define WQ_KVV_ALL(T)                                                                  \
+  switch (lpr) {                                                                       \
+    WQ_KVV(T, 1) WQ_KVV(T, 2) WQ_KVV(T, 4) WQ_KVV(T, 8) WQ_KVV(T, 16) WQ_KVV(T, 32) \
+    default: return WQ_ERR_ARG;                                                        \
+  }
+  switch (dtype) {
+    case WQ_F32: WQ_KVV_ALL(float); break;
+    case WQ_BF16: WQ_KVV_ALL(__nv_bfloat16); break;
+    default: WQ_KVV_ALL(__half); break;
+  }
+#undef WQ_KVV_ALL
+#undef WQ_KVV
+  WQ_LAUNCH_CHECK("kv_v_quant_kernel");
   return WQ_OK;
 }
 

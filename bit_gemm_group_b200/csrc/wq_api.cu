@@ -300,6 +300,24 @@ int wq_gemm_w8a8_smooth(const void* X, int64_t M, int64_t K, const void* Wq,
                                    Y, ws, acc_out, as_stream(stream));
 }
 
+// ---------------------------------------------------------------- KV cache
+
+int wq_quant_kv(const void* K, const void* V, int dtype, int64_t BH, int64_t S, int64_t D,
+                void* qk, void* sk, void* qv, void* sv, void* stream) {
+  if (BH < 0 || S < 0 || D < 0) return WQ_ERR_ARG;
+  if (dtype != WQ_F32 && dtype != WQ_BF16 && dtype != WQ_F16) return WQ_ERR_ARG;
+  if ((D % 8) != 0) return WQ_ERR_ALIGN;
+  if (D > 256 || BH > 65535) return WQ_ERR_UNSUPPORTED;
+  if (BH == 0 || D == 0) return WQ_OK;
+  if (!K || !V || !qk || !sk || !qv || !sv) return WQ_ERR_ARG;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(qk) || !aligned16(sk) || !aligned16(qv) ||
+      !aligned16(sv))
+    return WQ_ERR_ALIGN;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  return wq_host::launch_quant_kv(K, V, dtype, BH, S, D, qk, sk, qv, sv, as_stream(stream));
+}
+
 int wq_get_device_status(void* stream, int reset) {
   int st = wq_host::ensure_device();
   if (st != WQ_OK) return st;

@@ -244,6 +244,24 @@ WQ_API int wq_gemm_w8a8_smooth(const void *X, int64_t M, int64_t K, const void *
                                void *stream);
 
 /*
+ * wq_quant_kv -- KV-cache INT8 ([P4] sec. 6: K and V are treated differently).
+ * K, V [BH, S, D] of dtype (WQ_F32 / WQ_BF16 / WQ_F16), BH = batch x kv heads,
+ * S tokens, D head dim.
+ *   V per token:   sv[bh, t] = max(max_d |V[bh, t, d]| / 127, 1e-8),
+ *                  qv = clamp(round(V / sv), -128, 127)   (the page's
+ *                  quant_kv_per_token; same quantizer as wq_quant_act_i8)
+ *   K per channel: sk[bh, d] = max(max_t |K[bh, t, d]| / 127, 1e-8) over the
+ *                  S tokens of that head, qk = clamp(round(K / sk), -128, 127)
+ * qk, qv int8 [BH, S, D]; sk fp32 [BH, D]; sv fp32 [BH, S].  Rounding is half
+ * to even after one IEEE fp32 division.  Requires D % 8 == 0, D <= 256,
+ * BH <= 65535.  K is read twice (its channel maxima span all S tokens).
+ * Keeping the most recent tokens unquantized (the page's residual window) is
+ * the caller's choice of S.
+ */
+WQ_API int wq_quant_kv(const void *K, const void *V, int dtype, int64_t BH, int64_t S,
+                       int64_t D, void *qk, void *sk, void *qv, void *sv, void *stream);
+
+/*
  * wq_get_device_status -- synchronize `stream`, then return the first error
  * any kernel recorded since the last reset (WQ_OK if none); clear it when
  * reset != 0.  Returns WQ_ERR_CUDA if the synchronization itself fails.

@@ -117,3 +117,12 @@ def test_smoothquant_validation(L):
                                  None, None) == wq.WQ_ERR_ARG
     assert L.wq_gemm_w8a8_smooth(FAKE, 8, 128, FAKE, FAKE, FAKE, 16, FAKE, FAKE, 0,
                                  None, None) == wq.WQ_ERR_WORKSPACE
+
+
+def test_quant_kv_validation(L):
+    assert L.wq_quant_kv(FAKE, FAKE, 1, 2, 8, 12, FAKE, FAKE, FAKE, FAKE, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_quant_kv(FAKE, FAKE, 1, 2, 8, 264, FAKE, FAKE, FAKE, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_quant_kv(FAKE, FAKE, 5, 2, 8, 128, FAKE, FAKE, FAKE, FAKE, None) == wq.WQ_ERR_ARG
+    assert L.wq_quant_kv(FAKE, None, 1, 2, 8, 128, FAKE, FAKE, FAKE, FAKE, None) == wq.WQ_ERR_ARG
+    assert L.wq_quant_kv(FAKE, FAKE, 1, 70000, 8, 128, FAKE, FAKE, FAKE, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_quant_kv(FAKE, FAKE, 1, 0, 8, 128, FAKE, FAKE, FAKE, FAKE, None) == wq.WQ_OK
