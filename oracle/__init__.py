@@ -67,13 +67,20 @@ def _declare(L):
     L.oracle_quantize_int8_rows_smoothed.argtypes = [_P, _INT, _I64, _I64, _P, _P, _P]
     L.oracle_quant_act_i8_smoothed.argtypes = [_P, _INT, _I64, _I64, _P, _P, _P]
     L.oracle_quant_kv.argtypes = [_P, _P, _INT, _I64, _I64, _I64, _P, _P, _P, _P]
+    L.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+    L.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+    L.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+    L.oracle_e4m3_to_f32.restype = ctypes.c_float
+    L.oracle_quantize_fp8_rows.argtypes = [_P, _INT, _I64, _I64, _P, _P]
+    L.oracle_gemm_fp8.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _I64,
+                                  _P, _P]
     for name in ("oracle_quantize_int4", "oracle_quantize_int8_rows",
                  "oracle_quant_act_i8", "oracle_dequant_int4",
                  "oracle_dequant_int8_rows", "oracle_gemm_w4a16",
                  "oracle_gemm_w8a8_acc", "oracle_w8a8_rescale",
                  "oracle_channel_absmax", "oracle_smooth_scales",
                  "oracle_quantize_int8_rows_smoothed", "oracle_quant_act_i8_smoothed",
-                 "oracle_quant_kv"):
+                 "oracle_quant_kv", "oracle_quantize_fp8_rows", "oracle_gemm_fp8"):
         getattr(L, name).restype = _INT
 
 
@@ -222,6 +229,40 @@ def quant_kv(Kc, Vc, dtype_tag=None):
     st = lib().oracle_quant_kv(_ptr(Kc), _ptr(Vc), tag, BH, S, D, _ptr(qk), _ptr(sk), _ptr(qv),
                                _ptr(sv))
     return qk, sk, qv, sv, st
+
+
+def f32_to_e4m3(x):
+    x = np.asarray(x, np.float32).ravel()
+    return np.array([lib().oracle_f32_to_e4m3(float(v)) for v in x], np.uint8)
+
+
+def e4m3_to_f32(c):
+    c = np.asarray(c, np.uint8).ravel()
+    return np.array([lib().oracle_e4m3_to_f32(int(v)) for v in c], np.float32)
+
+
+def quantize_fp8_rows(W, dtype_tag=None):
+    """Per-row E4M3 (weights per output channel, activations per token).
+    Returns (q uint8 e4m3 codes [R, K], scales f32 [R], status)."""
+    W, tag = _tag_and_bits(W, dtype_tag)
+    R, K = W.shape
+    q = np.zeros((R, K), np.uint8)
+    s = np.zeros((R,), np.float32)
+    st = lib().oracle_quantize_fp8_rows(_ptr(W), tag, R, K, _ptr(q), _ptr(s))
+    return q, s, st
+
+
+def gemm_fp8(qx, sx, qw, sw, m0, m1, n0, n1):
+    """FP8 W8A8 product over a window: (Y fp64, exact fp64 sums, status)."""
+    qx = _c(qx, np.uint8); qw = _c(qw, np.uint8)
+    sx = _c(sx, np.float32); sw = _c(sw, np.float32)
+    M, K = qx.shape
+    N = qw.shape[0]
+    Y = np.zeros((m1 - m0, n1 - n0), np.float64)
+    acc = np.zeros((m1 - m0, n1 - n0), np.float64)
+    st = lib().oracle_gemm_fp8(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), M, N, K, m0, m1, n0, n1,
+                               _ptr(Y), _ptr(acc))
+    return Y, acc, st
 
 
 def dequant_int4(codes, scales, zeros, K, group_size=128, sym=True):

@@ -552,3 +552,81 @@ int oracle_quant_kv(const void *K, const void *V, int dtype, int64_t BH,
   }
   return status;
 }
+
+/* ------------------------------------------------------------------------- */
+/* FP8 E4M3                                                                   */
+/* ------------------------------------------------------------------------- */
+
+/* Encoding from the format: value = (-1)^s * 2^(e - 7) * (1 + m/8) for
+ * exponent field e in 1..15 (except e = 15, m = 7: NaN), and
+ * (-1)^s * 2^-6 * (m/8) for e = 0.  Rounding: nearest, ties to the even
+ * mantissa; magnitudes that round above 448 saturate to 448. */
+uint8_t oracle_f32_to_e4m3(float f) {
+  const uint8_t sign = signbit(f) ? 0x80 : 0x00;
+  if (isnan(f)) return (uint8_t)(sign | 0x7F);
+  float a = fabsf(f);
+  if (a >= 448.0f) return (uint8_t)(sign | 0x7E);
+  if (a < 0.015625f) {                       /* below 2^-6: subnormal, step 2^-9 */
+    const float m = oracle_round_half_even(a * 512.0f);   /* exact scaling */
+    return (uint8_t)(sign | (uint8_t)m);     /* m = 8 is the smallest normal, 0x08 */
+  }
+  int e = 0;
+  float t = a;
+  while (t >= 2.0f) { t *= 0.5f; ++e; }      /* exact: powers of two */
+  while (t < 1.0f) { t *= 2.0f; --e; }
+  float m = oracle_round_half_even((t - 1.0f) * 8.0f);   /* (t - 1) * 8 is exact */
+  if (m >= 8.0f) { m = 0.0f; ++e; }
+  const int field = e + 7;
+  uint8_t code = (uint8_t)((field << 3) | (int)m);
+  if (code > 0x7E) code = 0x7E;              /* saturate (448 = 0x7E) */
+  return (uint8_t)(sign | code);
+}
+
+float oracle_e4m3_to_f32(uint8_t c) {
+  const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  float v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) v = ldexpf((float)m / 8.0f, -6);
+  else v = ldexpf(1.0f + (float)m / 8.0f, e - 7);
+  return sign ? -v : v;
+}
+
+/* The W8A8 recipe of [P4] sec. 2.3 / 4.2 with E4M3 in place of int8: one scale
+ * per row (output channel or token) mapping the row's largest magnitude onto
+ * the largest finite E4M3 value, 448. */
+int oracle_quantize_fp8_rows(const void *W, int w_dtype, int64_t R, int64_t K,
+                             uint8_t *q, float *scales) {
+  if (R < 0 || K <= 0) return ORACLE_ERR_ARG;
+  int status = ORACLE_OK;
+  for (int64_t r = 0; r < R; ++r) {
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+      float x = load_elem(W, w_dtype, r * K + k);
+      if (!isfinite(x)) status = ORACLE_ERR_NONFINITE;
+      if (fabsf(x) > amax) amax = fabsf(x);
+    }
+    float s = amax / 448.0f;
+    if (s < 1e-8f) s = 1e-8f;
+    scales[r] = s;
+    for (int64_t k = 0; k < K; ++k) q[r * K + k] = oracle_f32_to_e4m3(load_elem(W, w_dtype, r * K + k) / s);
+  }
+  return status;
+}
+
+int oracle_gemm_fp8(const uint8_t *qx, const float *sx, const uint8_t *qw,
+                    const float *sw, int64_t M, int64_t N, int64_t K,
+                    int64_t m0, int64_t m1, int64_t n0, int64_t n1, double *Y,
+                    double *acc) {
+  if (m0 < 0 || m1 > M || n0 < 0 || n1 > N || m0 > m1 || n0 > n1 || K <= 0) return ORACLE_ERR_ARG;
+  const int64_t W = n1 - n0;
+  for (int64_t m = m0; m < m1; ++m) {
+    for (int64_t n = n0; n < n1; ++n) {
+      double sum = 0.0;
+      for (int64_t k = 0; k < K; ++k)
+        sum += (double)oracle_e4m3_to_f32(qx[m * K + k]) * (double)oracle_e4m3_to_f32(qw[n * K + k]);
+      if (acc) acc[(m - m0) * W + (n - n0)] = sum;
+      Y[(m - m0) * W + (n - n0)] = sum * (double)sx[m] * (double)sw[n];
+    }
+  }
+  return ORACLE_OK;
+}

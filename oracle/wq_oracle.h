@@ -19,8 +19,9 @@
  *        (per-group granularity), sec. 4 (metadata share)
  *   [P4] "27届大模型面试准备（十九）：模型量化全攻略" sec. 2.1 (affine quantization,
  *        min-max scale), 2.2 (per-group g=128, 4.25-bit), 3 (per-tensor worked
- *        example), 4.2 (SmoothQuant smoothing), 6 (per-token absmax quantizer,
- *        KV-cache: K per channel, V per token)
+ *        example), 2.3 (FP8 E4M3 as an 8-bit format), 4.2 (SmoothQuant
+ *        smoothing), 6 (per-token absmax quantizer, KV-cache: K per channel,
+ *        V per token)
  *
  * Status codes returned by the oracle functions.
  */
@@ -114,6 +115,22 @@ int oracle_quant_act_i8_smoothed(const void *X, int x_dtype, int64_t M,
 int oracle_quant_kv(const void *K, const void *V, int dtype, int64_t BH,
                     int64_t S, int64_t D, int8_t *qk, float *sk, int8_t *qv,
                     float *sv);
+
+/* FP8 E4M3 ([P4] sec. 2.3 naming table): 1 sign, 4 exponent (bias 7), 3
+ * mantissa bits, no infinities, S.1111.111 = NaN, largest finite 448.
+ * Round to nearest even, saturating to +-448. */
+uint8_t oracle_f32_to_e4m3(float f);
+float oracle_e4m3_to_f32(uint8_t c);
+/* FP8 W8A8 operands: per-output-channel (weights) or per-token (activations)
+ * s = max(amax / 448, 1e-8), q = e4m3(x / s). */
+int oracle_quantize_fp8_rows(const void *W, int w_dtype, int64_t R, int64_t K,
+                             uint8_t *q, float *scales);
+/* Y[m - m0, n - n0] = (sum_k e4m3(qx[m,k]) e4m3(qw[n,k])) * sx[m] * sw[n] in
+ * binary64; the sum of products is exact in binary64. */
+int oracle_gemm_fp8(const uint8_t *qx, const float *sx, const uint8_t *qw,
+                    const float *sw, int64_t M, int64_t N, int64_t K,
+                    int64_t m0, int64_t m1, int64_t n0, int64_t n1, double *Y,
+                    double *acc);
 
 /* W8A8 rescale in fp64: Y = acc * sx[m] * sw[n] over the same window. */
 int oracle_w8a8_rescale(const int32_t *acc, const float *sx, const float *sw,
