@@ -451,6 +451,23 @@ def secondary(wq, dev, args):
     del qw, sw, X8, Y8, ws8, W8, s8, qws, sws
     torch.cuda.empty_cache()
 
+    # FP8 E4M3 W8A8 on the same workload (tcgen05.mma kind::f8f6f4)
+    W8 = wl8.weight(0).to(dev)
+    X8 = wl8.activation(4096, 4096).to(dev)
+    Y8 = torch.empty((4096, 4096), dtype=torch.bfloat16, device=dev)
+    ws8 = torch.empty((wq.wq_w8a8_workspace_bytes(4096, 4096),), dtype=torch.uint8, device=dev)
+    fw, fsw = wq.quantize_fp8_rows(W8)
+    t = time_flushed(lambda: wq.wq_gemm_fp8(X8, fw, fsw, Y8, ws8), flush)
+    fp8_peak = 2.0 * pk["bf16_tflops"]  # measured bf16 peak x the nominal fp8/bf16 ratio
+    out["fp8_tflops"] = round(ops / (t * 1e-3) / 1e12, 1)
+    out["fp8_us"] = round(t * 1e3, 1)
+    out["fp8_frac_peak"] = round(ops / (t * 1e-3) / 1e12 / fp8_peak, 3)
+    ref = X8[:256].double().cpu().numpy() @ W8.double().cpu().numpy().T
+    y8 = wq.gemm_fp8(X8[:256].contiguous(), fw, fsw).double().cpu().numpy()
+    out["fp8_rel_err"] = float(f"{np.linalg.norm(y8 - ref) / np.linalg.norm(ref):.3e}")
+    del W8, X8, Y8, ws8, fw, fsw
+    torch.cuda.empty_cache()
+
     # KV-cache INT8 (K per channel, V per token), bf16 cache of 8 kv heads x 8
     # sequences x 8192 tokens x 128 dims (2 x 134 MB, larger than L2).  The
     # algorithmic bytes count one read of K and V, the int8 writes and the

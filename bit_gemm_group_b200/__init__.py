@@ -40,7 +40,7 @@ EXPORTED = (
     "wq_status_str", "wq_last_cuda_error", "wq_selftest_wait_timeout",
     "wq_gemm_w4a16_noalloc",
     "wq_channel_absmax", "wq_smooth_scales", "wq_quantize_i8_smooth", "wq_quant_act_i8_smooth",
-    "wq_gemm_w8a8_smooth", "wq_quant_kv",
+    "wq_gemm_w8a8_smooth", "wq_quant_kv", "wq_quantize_fp8_rows", "wq_gemm_fp8",
 )
 
 
@@ -107,10 +107,12 @@ def _declare(L):
     L.wq_quant_act_i8_smooth.argtypes = [_P, _I64, _I64, _P, _P, _P, _P]
     L.wq_gemm_w8a8_smooth.argtypes = [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _SZ, _P, _P]
     L.wq_quant_kv.argtypes = [_P, _P, _INT, _I64, _I64, _I64, _P, _P, _P, _P, _P]
+    L.wq_quantize_fp8_rows.argtypes = [_P, _INT, _I64, _I64, _P, _P, _P]
+    L.wq_gemm_fp8.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P, _P, _SZ, _P, _P]
     for name in ("wq_quantize_pack", "wq_dequant", "wq_gemm_w4a16", "wq_quant_act_i8",
                  "wq_gemm_w8a8", "wq_get_device_status", "wq_channel_absmax",
                  "wq_smooth_scales", "wq_quantize_i8_smooth", "wq_quant_act_i8_smooth",
-                 "wq_gemm_w8a8_smooth", "wq_quant_kv"):
+                 "wq_gemm_w8a8_smooth", "wq_quant_kv", "wq_quantize_fp8_rows", "wq_gemm_fp8"):
         getattr(L, name).restype = _INT
 
 
@@ -247,6 +249,21 @@ def wq_quant_kv(K, V, qk, sk, qv, sv, stream=None):
     _check(st, "wq_quant_kv")
 
 
+def wq_quantize_fp8_rows(A, q, scales, stream=None):
+    R, K = A.shape
+    st = lib().wq_quantize_fp8_rows(_ptr(A), _DTYPE_TAG.get(A.dtype, -1), R, K, _ptr(q),
+                                    _ptr(scales), _stream(stream))
+    _check(st, "wq_quantize_fp8_rows")
+
+
+def wq_gemm_fp8(X, Wq, w_scales, Y, ws, acc_out=None, stream=None):
+    M, K = X.shape
+    N = Wq.shape[0]
+    st = lib().wq_gemm_fp8(_ptr(X), M, K, _ptr(Wq), _ptr(w_scales), N, _ptr(Y), _ptr(ws),
+                           ws.numel() * ws.element_size(), _ptr(acc_out), _stream(stream))
+    _check(st, "wq_gemm_fp8")
+
+
 def wq_get_device_status(reset=True, stream=None):
     """Synchronize the stream and return the first kernel-detected error code."""
     return int(lib().wq_get_device_status(_stream(stream), int(bool(reset))))
@@ -379,3 +396,25 @@ def quant_kv(K, V):
     sv = torch.empty((BH, S), dtype=torch.float32, device=K.device)
     wq_quant_kv(K, V, qk, sk, qv, sv)
     return qk, sk, qv, sv
+
+
+# ------------------------------------------------------------------ FP8 helpers
+
+def quantize_fp8_rows(A):
+    """Per-row E4M3: (codes uint8 [R, K], scales fp32 [R])."""
+    R, K = A.shape
+    q = torch.empty((R, K), dtype=torch.uint8, device=A.device)
+    s = torch.empty((R,), dtype=torch.float32, device=A.device)
+    wq_quantize_fp8_rows(A, q, s)
+    return q, s
+
+
+def gemm_fp8(X, Wq, w_scales, want_acc=False):
+    M, K = X.shape
+    N = Wq.shape[0]
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    ws = torch.empty((max(1, wq_w8a8_workspace_bytes(M, K)),), dtype=torch.uint8,
+                     device=X.device)
+    acc = torch.empty((M, N), dtype=torch.float32, device=X.device) if want_acc else None
+    wq_gemm_fp8(X, Wq, w_scales, Y, ws, acc)
+    return (Y, acc) if want_acc else Y

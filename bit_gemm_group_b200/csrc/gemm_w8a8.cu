@@ -26,6 +26,7 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 512;  // two 128 x 256 int32 accumulators
 constexpr int THREADS = 192;
 constexpr uint32_t IDESC = tc::idesc_s8_s32(BM, BN);
+constexpr uint32_t IDESC_FP8 = tc::idesc_e4m3_f32(BM, BN);
 
 struct Smem {
   uint64_t full[STAGES];
@@ -38,10 +39,14 @@ struct Smem {
 };
 constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + size_t(STAGES) * STAGE_BYTES + sizeof(Smem);
 
+// FP8 = false: int8 operands, tcgen05.mma kind::i8, int32 accumulators;
+// FP8 = true: E4M3 operands, kind::f8f6f4, fp32 accumulators (same tiles,
+// same 32-element K steps, same epilogue up to the accumulator type).
+template <bool FP8>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const float* __restrict__ sx, const float* __restrict__ sw,
-                     __nv_bfloat16* __restrict__ Y, int32_t* __restrict__ acc_out, int M, int N,
+                     __nv_bfloat16* __restrict__ Y, uint32_t* __restrict__ acc_out, int M, int N,
                      int K, int* status, uint64_t limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -124,9 +129,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t a = tc::smem_u32(tiles + size_t(s) * STAGE_BYTES);
           const uint32_t b = a + A_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / 32; ++k)
-            tc::mma_i8_ss(d, tc::sdesc_k_sw128(a + k * 32), tc::sdesc_k_sw128(b + k * 32), IDESC,
-                          (kb | k) != 0);
+          for (int k = 0; k < BK / 32; ++k) {
+            if (FP8)
+              tc::mma_f8_ss(d, tc::sdesc_k_sw128(a + k * 32), tc::sdesc_k_sw128(b + k * 32),
+                            IDESC_FP8, (kb | k) != 0);
+            else
+              tc::mma_i8_ss(d, tc::sdesc_k_sw128(a + k * 32), tc::sdesc_k_sw128(b + k * 32),
+                            IDESC, (kb | k) != 0);
+          }
           tc::mma_commit(&sm.empty[s]);
         }
         if (ok) tc::mma_commit(&sm.tfull[buf]);
@@ -164,14 +174,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             } o;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float v0 = float(int32_t(r[g * 8 + 2 * j])) * srow * __ldg(sw + n + 2 * j);
-              const float v1 =
-                  float(int32_t(r[g * 8 + 2 * j + 1])) * srow * __ldg(sw + n + 2 * j + 1);
+              const uint32_t a0 = r[g * 8 + 2 * j], a1 = r[g * 8 + 2 * j + 1];
+              const float f0 = FP8 ? __uint_as_float(a0) : float(int32_t(a0));
+              const float f1 = FP8 ? __uint_as_float(a1) : float(int32_t(a1));
+              const float v0 = f0 * srow * __ldg(sw + n + 2 * j);
+              const float v1 = f1 * srow * __ldg(sw + n + 2 * j + 1);
               o.h[j] = __floats2bfloat162_rn(v0, v1);
             }
             *reinterpret_cast<uint4*>(Y + size_t(row) * N + n) = o.v;
             if (acc_out != nullptr) {
-              int32_t* dst = acc_out + size_t(row) * N + n;
+              uint32_t* dst = acc_out + size_t(row) * N + n;
               reinterpret_cast<uint4*>(dst)[0] =
                   make_uint4(r[g * 8 + 0], r[g * 8 + 1], r[g * 8 + 2], r[g * 8 + 3]);
               reinterpret_cast<uint4*>(dst)[1] =
@@ -198,40 +210,68 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 namespace wq_host {
 
-int launch_gemm_w8a8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
-                     const float* smooth, int64_t N, void* Y, void* ws, void* acc_out,
-                     cudaStream_t s) {
+static int launch_gemm_8bit(bool fp8, const void* qx, const float* sx, int64_t M, int64_t K,
+                            const void* Wq, const void* w_scales, int64_t N, void* Y,
+                            void* acc_out, cudaStream_t s) {
   using namespace wq::w8a8;
-  int8_t* qx = static_cast<int8_t*>(ws);
-  float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
-                                       ((size_t(M) * size_t(K) + 255) & ~size_t(255)));
-  int st = launch_quantize_rows_i8(X, WQ_BF16, M, K, true, smooth, qx, sx, s);
-  if (st != WQ_OK) return st;
-
   CUtensorMap ta, tb;
-  st = make_tmap_2d(&ta, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(M), uint64_t(K), BM, BK,
-                    128);
+  int st = make_tmap_2d(&ta, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(M), uint64_t(K), BM, BK,
+                        128);
   if (st != WQ_OK) return st;
   st = make_tmap_2d(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(N), uint64_t(K), BN, BK,
                     128);
   if (st != WQ_OK) return st;
 
-  static bool attr_done[64] = {};
+  static bool attr_done[2][64] = {};
   int dev = 0;
   WQ_CUDA_CHECK(cudaGetDevice(&dev));
-  if (dev < 64 && !attr_done[dev]) {
-    WQ_CUDA_CHECK(cudaFuncSetAttribute(gemm_w8a8_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(SMEM_BYTES)));
-    attr_done[dev] = true;
+  if (dev < 64 && !attr_done[fp8][dev]) {
+    if (fp8)
+      WQ_CUDA_CHECK(cudaFuncSetAttribute(gemm_w8a8_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(SMEM_BYTES)));
+    else
+      WQ_CUDA_CHECK(cudaFuncSetAttribute(gemm_w8a8_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(SMEM_BYTES)));
+    attr_done[fp8][dev] = true;
   }
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = int(tiles < sm_count() ? tiles : sm_count());
-  gemm_w8a8_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(
-      ta, tb, sx, static_cast<const float*>(w_scales), static_cast<__nv_bfloat16*>(Y),
-      static_cast<int32_t*>(acc_out), int(M), int(N), int(K), status_ptr(), wait_limit_ns());
+  auto* y = static_cast<__nv_bfloat16*>(Y);
+  auto* acc = static_cast<uint32_t*>(acc_out);
+  auto* sw = static_cast<const float*>(w_scales);
+  if (fp8)
+    gemm_w8a8_kernel<true><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, sx, sw, y, acc, int(M),
+                                                             int(N), int(K), status_ptr(),
+                                                             wait_limit_ns());
+  else
+    gemm_w8a8_kernel<false><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, sx, sw, y, acc, int(M),
+                                                              int(N), int(K), status_ptr(),
+                                                              wait_limit_ns());
   WQ_LAUNCH_CHECK("gemm_w8a8_kernel");
   return WQ_OK;
+}
+
+int launch_gemm_w8a8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
+                     const float* smooth, int64_t N, void* Y, void* ws, void* acc_out,
+                     cudaStream_t s) {
+  int8_t* qx = static_cast<int8_t*>(ws);
+  float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                       ((size_t(M) * size_t(K) + 255) & ~size_t(255)));
+  int st = launch_quantize_rows_i8(X, WQ_BF16, M, K, true, smooth, qx, sx, s);
+  if (st != WQ_OK) return st;
+  return launch_gemm_8bit(false, qx, sx, M, K, Wq, w_scales, N, Y, acc_out, s);
+}
+
+int launch_gemm_fp8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
+                    int64_t N, void* Y, void* ws, void* acc_out, cudaStream_t s) {
+  uint8_t* qx = static_cast<uint8_t*>(ws);
+  float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                       ((size_t(M) * size_t(K) + 255) & ~size_t(255)));
+  int st = launch_quantize_rows_fp8(X, WQ_BF16, M, K, qx, sx, s);
+  if (st != WQ_OK) return st;
+  return launch_gemm_8bit(true, qx, sx, M, K, Wq, w_scales, N, Y, acc_out, s);
 }
 
 }  // namespace wq_host

@@ -19,6 +19,10 @@ int launch_smooth_scales(const float* act, const float* w, int64_t K, float alph
                          cudaStream_t s);
 int launch_quant_kv(const void* Kc, const void* Vc, int dtype, int64_t BH, int64_t S, int64_t D,
                     void* qk, void* sk, void* qv, void* sv, cudaStream_t s);
+int launch_quantize_rows_fp8(const void* W, int w_dtype, int64_t R, int64_t K, void* q,
+                             void* scales, cudaStream_t s);
+int launch_gemm_fp8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
+                    int64_t N, void* Y, void* ws, void* acc_out, cudaStream_t s);
 int launch_dequant_int4(const void* codes, const void* scales, const void* zeros, int64_t N,
                         int64_t K, int group_size, int sym, void* out, int out_dtype,
                         cudaStream_t s);

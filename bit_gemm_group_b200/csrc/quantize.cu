@@ -10,6 +10,7 @@
 // grid as a multiple of the SM count.
 #include "common.cuh"
 #include "kernels.h"
+#include <cuda_fp8.h>
 
 namespace wq {
 
@@ -235,6 +236,66 @@ __global__ void __launch_bounds__(256) quantize_rows_i8_kernel(
         }
         o.b[e] = int8_t(qi);
       }
+      *reinterpret_cast<uint2*>(q + r * K + k) = o.v2;
+    }
+    __syncthreads();  // red[] is reused by the next row
+  }
+}
+
+// ---------------------------------------------------------------------------
+// FP8 E4M3 rows ("27届大模型面试准备（十九）…" sec. 2.3: FP8 as the 8-bit float
+// format; the W8A8 recipe with E4M3 in place of int8)
+// ---------------------------------------------------------------------------
+// One scale per row, s = max(amax / 448, 1e-8), q = e4m3(x / s) rounded to
+// nearest even and saturated to +-448 (the hardware conversion).
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(
+    const T* __restrict__ X, int64_t rows, int64_t K, uint8_t* __restrict__ q,
+    float* __restrict__ scales, int* status) {
+  constexpr int EV = 8;
+  __shared__ float red[8];
+  __shared__ int bad_any;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const T* row = X + r * K;
+    float amax = 0.f;
+    bool finite = true;
+    for (int64_t k = int64_t(threadIdx.x) * EV; k < K; k += int64_t(blockDim.x) * EV) {
+      Elems<T, EV> v;
+      v.load(row + k);
+#pragma unroll
+      for (int e = 0; e < EV; ++e) {
+        const float x = to_f32<T>(v.u.e[e]);
+        finite &= isfinite(x);
+        amax = fmaxf(amax, fabsf(x));
+      }
+    }
+    amax = warp_max(amax);
+    const int nbad = __syncthreads_or(!finite);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float m = red[0];
+      for (int w = 1; w < int(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+      red[0] = m;
+      bad_any = nbad;
+    }
+    __syncthreads();
+    const float s = fmaxf(div_rn(red[0], 448.f), 1e-8f);
+    if (threadIdx.x == 0) {
+      scales[r] = s;
+      if (bad_any) record_error(status, WQ_ERR_NONFINITE);
+    }
+    for (int64_t k = int64_t(threadIdx.x) * EV; k < K; k += int64_t(blockDim.x) * EV) {
+      Elems<T, EV> v;
+      v.load(row + k);
+      union {
+        uint2 v2;
+        uint8_t b[EV];
+      } o;
+#pragma unroll
+      for (int e = 0; e < EV; ++e)
+        o.b[e] = uint8_t(__nv_cvt_float_to_fp8(div_rn(to_f32<T>(v.u.e[e]), s), __NV_SATFINITE,
+                                               __NV_E4M3));
       *reinterpret_cast<uint2*>(q + r * K + k) = o.v2;
     }
     __syncthreads();  // red[] is reused by the next row
@@ -587,6 +648,31 @@ int launch_quantize_rows_i8(const void* W, int w_dtype, int64_t N, int64_t K, bo
   }
 #undef WQ_ROWS
   WQ_LAUNCH_CHECK("quantize_rows_i8_kernel");
+  return WQ_OK;
+}
+
+int launch_quantize_rows_fp8(const void* W, int w_dtype, int64_t R, int64_t K, void* q,
+                             void* scales, cudaStream_t s) {
+  const int grid = int(R < int64_t(sm_count()) * 16 ? R : int64_t(sm_count()) * 16);
+  int* st = status_ptr();
+  auto* qo = static_cast<uint8_t*>(q);
+  auto* so = static_cast<float*>(scales);
+  switch (w_dtype) {
+    case WQ_F32:
+      wq::quantize_rows_fp8_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(W), R, K,
+                                                               qo, so, st);
+      break;
+    case WQ_BF16:
+      wq::quantize_rows_fp8_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(W), R, K, qo, so, st);
+      break;
+    case WQ_F16:
+      wq::quantize_rows_fp8_kernel<__half><<<grid, 256, 0, s>>>(static_cast<const __half*>(W), R,
+                                                                K, qo, so, st);
+      break;
+    default: return WQ_ERR_ARG;
+  }
+  WQ_LAUNCH_CHECK("quantize_rows_fp8_kernel");
   return WQ_OK;
 }
 

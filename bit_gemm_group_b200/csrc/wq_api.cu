@@ -318,6 +318,39 @@ int wq_quant_kv(const void* K, const void* V, int dtype, int64_t BH, int64_t S, 
   return wq_host::launch_quant_kv(K, V, dtype, BH, S, D, qk, sk, qv, sv, as_stream(stream));
 }
 
+// --------------------------------------------------------------------- FP8
+
+int wq_quantize_fp8_rows(const void* A, int a_dtype, int64_t R, int64_t K, void* q, void* scales,
+                         void* stream) {
+  if (R < 0 || K < 0) return WQ_ERR_ARG;
+  if (a_dtype != WQ_F32 && a_dtype != WQ_BF16 && a_dtype != WQ_F16) return WQ_ERR_ARG;
+  if ((K % 16) != 0) return WQ_ERR_ALIGN;
+  if (R == 0 || K == 0) return WQ_OK;
+  if (!A || !q || !scales) return WQ_ERR_ARG;
+  if (!aligned16(A) || !aligned16(q) || !aligned16(scales)) return WQ_ERR_ALIGN;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  return wq_host::launch_quantize_rows_fp8(A, a_dtype, R, K, q, scales, as_stream(stream));
+}
+
+int wq_gemm_fp8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
+                int64_t N, void* Y, void* ws, size_t ws_bytes, void* acc_out, void* stream) {
+  if (M < 0 || K < 0 || N < 0) return WQ_ERR_ARG;
+  if ((K % 16) != 0 || (N % 16) != 0) return WQ_ERR_ALIGN;
+  if (M > (int64_t(1) << 31) / 2 || N > (int64_t(1) << 31) / 2 || K > (int64_t(1) << 24))
+    return WQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return WQ_OK;
+  if (K == 0) return WQ_ERR_ARG;
+  if (!X || !Wq || !w_scales || !Y) return WQ_ERR_ARG;
+  if (!ws || ws_bytes < wq_w8a8_workspace_bytes(M, K)) return WQ_ERR_WORKSPACE;
+  if (!aligned16(X) || !aligned16(Wq) || !aligned16(w_scales) || !aligned16(Y) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || (acc_out && !aligned16(acc_out)))
+    return WQ_ERR_ALIGN;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  return wq_host::launch_gemm_fp8(X, M, K, Wq, w_scales, N, Y, ws, acc_out, as_stream(stream));
+}
+
 int wq_get_device_status(void* stream, int reset) {
   int st = wq_host::ensure_device();
   if (st != WQ_OK) return st;

@@ -262,6 +262,33 @@ WQ_API int wq_quant_kv(const void *K, const void *V, int dtype, int64_t BH, int6
                        int64_t D, void *qk, void *sk, void *qv, void *sv, void *stream);
 
 /*
+ * FP8 E4M3 W8A8 ([P4] sec. 2.3 names FP8 E4M3 as the 8-bit float format of
+ * the newest tensor cores; the recipe is the W8A8 one with E4M3 in place of
+ * int8).  E4M3: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, largest
+ * finite value 448, no infinities.
+ *
+ * wq_quantize_fp8_rows -- one scale per row (a weight's output channel, or an
+ * activation's token): s[r] = max(max_k |A[r, k]| / 448, 1e-8) and
+ * q = E4M3(A / s) (IEEE division, round to nearest even, saturating to
+ * +-448).  A [R, K] of a_dtype -> q uint8 E4M3 codes [R, K], s fp32 [R].
+ * Requires K % 16 == 0.
+ */
+WQ_API int wq_quantize_fp8_rows(const void *A, int a_dtype, int64_t R, int64_t K,
+                                void *q, void *scales, void *stream);
+
+/*
+ * wq_gemm_fp8 -- Y = bf16(acc * sx[m] * w_scales[n]) with acc[m, n] =
+ * sum_k E4M3(qx[m, k]) * E4M3(qw[n, k]) accumulated in fp32 on the tensor cores
+ * (tcgen05.mma kind::f8f6f4).  X bf16 [M, K] is quantized per token into ws
+ * first (as wq_quantize_fp8_rows); Wq / w_scales come from
+ * wq_quantize_fp8_rows on the weight.  acc_out (nullable) receives the fp32
+ * accumulators [M, N].  Same requirements and workspace as wq_gemm_w8a8.
+ */
+WQ_API int wq_gemm_fp8(const void *X, int64_t M, int64_t K, const void *Wq,
+                       const void *w_scales, int64_t N, void *Y, void *ws,
+                       size_t ws_bytes, void *acc_out, void *stream);
+
+/*
  * wq_get_device_status -- synchronize `stream`, then return the first error
  * any kernel recorded since the last reset (WQ_OK if none); clear it when
  * reset != 0.  Returns WQ_ERR_CUDA if the synchronization itself fails.

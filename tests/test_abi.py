@@ -126,3 +126,12 @@ def test_quant_kv_validation(L):
     assert L.wq_quant_kv(FAKE, None, 1, 2, 8, 128, FAKE, FAKE, FAKE, FAKE, None) == wq.WQ_ERR_ARG
     assert L.wq_quant_kv(FAKE, FAKE, 1, 70000, 8, 128, FAKE, FAKE, FAKE, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
     assert L.wq_quant_kv(FAKE, FAKE, 1, 0, 8, 128, FAKE, FAKE, FAKE, FAKE, None) == wq.WQ_OK
+
+
+def test_fp8_validation(L):
+    assert L.wq_quantize_fp8_rows(FAKE, 1, 8, 24, FAKE, FAKE, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_quantize_fp8_rows(FAKE, 4, 8, 32, FAKE, FAKE, None) == wq.WQ_ERR_ARG
+    assert L.wq_quantize_fp8_rows(FAKE, 1, 0, 32, FAKE, FAKE, None) == wq.WQ_OK
+    assert L.wq_gemm_fp8(FAKE, 8, 128, FAKE, FAKE, 24, FAKE, FAKE, 1 << 20, None, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_gemm_fp8(FAKE, 8, 128, FAKE, FAKE, 16, FAKE, FAKE, 0, None, None) == wq.WQ_ERR_WORKSPACE
+    assert L.wq_gemm_fp8(FAKE, 8, 128, None, FAKE, 16, FAKE, FAKE, 1 << 20, None, None) == wq.WQ_ERR_ARG
