@@ -212,6 +212,20 @@ def time_flushed(fn, flush, reps=10, warm=3):
 
 # ----------------------------------------------------------------- our arm
 
+def job_time_ms(local_ms, world, device):
+    """The job's time: the slowest rank's device time (all ranks take part)."""
+    if world <= 1:
+        return float(local_ms)
+    tt = torch.tensor([float(local_ms)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_throughput_gbs(world, steps, step_bytes, ms):
+    """Whole-job GB/s: every rank streams its own replica's bytes each step."""
+    return world * steps * step_bytes / (ms * 1e-3) / 1e9
+
+
 def run_ours(args, rank, world, local_rank):
     import bit_gemm_group_b200 as wq
 
@@ -264,11 +278,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     sampler.stop()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = job_time_ms(t0.elapsed_time(t1), world, dev)
     clocks = sampler.summary(mark)
 
     # kernel time per shape from the events around each graph replay
@@ -277,7 +287,7 @@ def run_ours(args, rank, world, local_rank):
     launches_timed = (args.steps // ROT) * ROT
     kernel_total_ms = sum(kern_ms)
     pk = peaks()
-    value = world * args.steps * step_bytes / (ms * 1e-3) / 1e9
+    value = job_throughput_gbs(world, args.steps, step_bytes, ms)
     achieved = (launches_timed * step_bytes / (kernel_total_ms * 1e-3) / 1e9
                 if kernel_total_ms > 0 else None)
 
