@@ -74,13 +74,16 @@ def _declare(L):
     L.oracle_quantize_fp8_rows.argtypes = [_P, _INT, _I64, _I64, _P, _P]
     L.oracle_gemm_fp8.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _I64,
                                   _P, _P]
+    L.oracle_gptq_hinv_chol.argtypes = [_P, _INT, _I64, _I64, ctypes.c_double, _P]
+    L.oracle_gptq_quantize.argtypes = [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P]
     for name in ("oracle_quantize_int4", "oracle_quantize_int8_rows",
                  "oracle_quant_act_i8", "oracle_dequant_int4",
                  "oracle_dequant_int8_rows", "oracle_gemm_w4a16",
                  "oracle_gemm_w8a8_acc", "oracle_w8a8_rescale",
                  "oracle_channel_absmax", "oracle_smooth_scales",
                  "oracle_quantize_int8_rows_smoothed", "oracle_quant_act_i8_smoothed",
-                 "oracle_quant_kv", "oracle_quantize_fp8_rows", "oracle_gemm_fp8"):
+                 "oracle_quant_kv", "oracle_quantize_fp8_rows", "oracle_gemm_fp8",
+                 "oracle_gptq_hinv_chol", "oracle_gptq_quantize"):
         getattr(L, name).restype = _INT
 
 
@@ -263,6 +266,29 @@ def gemm_fp8(qx, sx, qw, sw, m0, m1, n0, n1):
     st = lib().oracle_gemm_fp8(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), M, N, K, m0, m1, n0, n1,
                                _ptr(Y), _ptr(acc))
     return Y, acc, st
+
+
+def gptq_hinv_chol(X, damp=0.01, dtype_tag=None):
+    """GPTQ factor U [K, K] (fp64, upper) of H^-1, H = 2 X^T X + damp mean(diag H) I."""
+    X, tag = _tag_and_bits(X, dtype_tag)
+    T, K = X.shape
+    U = np.zeros((K, K), np.float64)
+    st = lib().oracle_gptq_hinv_chol(_ptr(X), tag, T, K, float(damp), _ptr(U))
+    return U, st
+
+
+def gptq_quantize(W, U, group_size=128, sym=True, dtype_tag=None):
+    """GPTQ INT4: (codes u8 [N, K/2], scales f16 bits [N, G], zeros f16 bits or None, status)."""
+    W, tag = _tag_and_bits(W, dtype_tag)
+    N, K = W.shape
+    U = _c(U, np.float64)
+    G = K // group_size
+    codes = np.zeros((N, K // 2), np.uint8)
+    scales = np.zeros((N, G), np.uint16)
+    zeros = None if sym else np.zeros((N, G), np.uint16)
+    st = lib().oracle_gptq_quantize(_ptr(W), tag, N, K, _ptr(U), group_size, int(bool(sym)),
+                                    _ptr(codes), _ptr(scales), _ptr(zeros))
+    return codes, scales, zeros, st
 
 
 def dequant_int4(codes, scales, zeros, K, group_size=128, sym=True):

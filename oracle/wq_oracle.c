@@ -187,6 +187,54 @@ static int clamp_int(int v, int lo, int hi) {
  *     byte, element k of row n in byte n*K/2 + k/2, low nibble = even k;
  *     zero points are stored as fp16 integers 0..15 (asym only).
  */
+/* Scale (fp16 bits), zero point and degeneracy of one group of n values
+ * ([P3] sec. 2.1 / [P4] sec. 2.1, readings in the header): sym s = amax/7,
+ * asym s = (max - min)/15 and z = clamp(round(-min/s), 0, 15); the fp32
+ * scale is rounded to fp16 and the fp16 value is the one used. */
+static void group_params(const float *x, int64_t n, int sym, uint16_t *s16_out,
+                         int *z_out, int *degenerate_out, int *nonfinite) {
+  float mn = INFINITY, mx = -INFINITY, amax = 0.0f;
+  for (int64_t k = 0; k < n; ++k) {
+    if (!isfinite(x[k])) *nonfinite = 1;
+    if (x[k] < mn) mn = x[k];
+    if (x[k] > mx) mx = x[k];
+    if (fabsf(x[k]) > amax) amax = fabsf(x[k]);
+  }
+  uint16_t s16;
+  int z = 0;
+  int degenerate;
+  if (sym) {
+    float s32 = amax / 7.0f;
+    s16 = oracle_f32_to_f16(s32);
+    degenerate = (amax < 1e-8f) || (oracle_f16_to_f32(s16) == 0.0f);
+    if (degenerate) s16 = oracle_f32_to_f16(amax);
+  } else {
+    float range = mx - mn;
+    float s32 = range / 15.0f;
+    s16 = oracle_f32_to_f16(s32);
+    degenerate = (range < 1e-8f) || (oracle_f16_to_f32(s16) == 0.0f);
+    if (degenerate) {
+      s16 = oracle_f32_to_f16(1.0f);
+      z = 0;
+    } else {
+      float sf = oracle_f16_to_f32(s16);
+      float zr = oracle_round_half_even(-mn / sf);
+      z = (int)fmaxf(0.0f, fminf(15.0f, zr));
+    }
+  }
+  *s16_out = s16;
+  *z_out = z;
+  *degenerate_out = degenerate;
+}
+
+static void put_nibble(uint8_t *codes, int64_t idx, uint8_t u) {
+  uint8_t *byte = &codes[idx / 2];
+  if ((idx & 1) == 0)
+    *byte = (uint8_t)((*byte & 0xF0u) | u);
+  else
+    *byte = (uint8_t)((*byte & 0x0Fu) | (uint8_t)(u << 4));
+}
+
 int oracle_quantize_int4(const void *W, int w_dtype, int64_t N, int64_t K,
                          int group_size, int sym, uint8_t *codes,
                          uint16_t *scales, uint16_t *zeros) {
@@ -198,64 +246,36 @@ int oracle_quantize_int4(const void *W, int w_dtype, int64_t N, int64_t K,
   const int64_t G = K / group_size;
   const int qmin = sym ? -8 : 0;
   const int qmax = sym ? 7 : 15;
+  float *grp = (float *)malloc((size_t)group_size * sizeof(float));
+  if (!grp) return ORACLE_ERR_ARG;
   memset(codes, 0, (size_t)(N * (K / 2)));
   for (int64_t n = 0; n < N; ++n) {
     for (int64_t g = 0; g < G; ++g) {
       const int64_t k0 = g * group_size;
-      float mn = INFINITY, mx = -INFINITY, amax = 0.0f;
-      for (int64_t k = k0; k < k0 + group_size; ++k) {
-        float x = load_elem(W, w_dtype, n * K + k);
-        if (!isfinite(x)) status = ORACLE_ERR_NONFINITE;
-        if (x < mn) mn = x;
-        if (x > mx) mx = x;
-        if (fabsf(x) > amax) amax = fabsf(x);
-      }
+      for (int64_t k = 0; k < group_size; ++k) grp[k] = load_elem(W, w_dtype, n * K + k0 + k);
       uint16_t s16;
-      int z = 0;
-      int degenerate;
-      if (sym) {
-        float s32 = amax / 7.0f;
-        s16 = oracle_f32_to_f16(s32);
-        degenerate = (amax < 1e-8f) || (oracle_f16_to_f32(s16) == 0.0f);
-        if (degenerate) s16 = oracle_f32_to_f16(amax);
-      } else {
-        float range = mx - mn;
-        float s32 = range / 15.0f;
-        s16 = oracle_f32_to_f16(s32);
-        degenerate = (range < 1e-8f) || (oracle_f16_to_f32(s16) == 0.0f);
-        if (degenerate) {
-          s16 = oracle_f32_to_f16(1.0f);
-          z = 0;
-        } else {
-          float sf = oracle_f16_to_f32(s16);
-          float zr = oracle_round_half_even(-mn / sf);
-          z = (int)fmaxf(0.0f, fminf(15.0f, zr));
-        }
-        zeros[n * G + g] = oracle_f32_to_f16((float)z);
-      }
+      int z, degenerate, nonfinite = 0;
+      group_params(grp, group_size, sym, &s16, &z, &degenerate, &nonfinite);
+      if (nonfinite) status = ORACLE_ERR_NONFINITE;
+      if (!sym) zeros[n * G + g] = oracle_f32_to_f16((float)z);
       if (isinf(oracle_f16_to_f32(s16))) status = ORACLE_ERR_NONFINITE;
       scales[n * G + g] = s16;
       const float sf = oracle_f16_to_f32(s16);
-      for (int64_t k = k0; k < k0 + group_size; ++k) {
+      for (int64_t k = 0; k < group_size; ++k) {
         int q;
         if (degenerate) {
           q = 0;
         } else {
-          float x = load_elem(W, w_dtype, n * K + k);
-          float r = oracle_round_half_even(x / sf);
+          float r = oracle_round_half_even(grp[k] / sf);
           /* clamp in float first so huge quotients do not overflow int */
           r = fmaxf(-64.0f, fminf(64.0f, r));
           q = clamp_int((int)r + z, qmin, qmax);
         }
-        uint8_t u = (uint8_t)(q - qmin);
-        uint8_t *byte = &codes[n * (K / 2) + k / 2];
-        if ((k & 1) == 0)
-          *byte = (uint8_t)((*byte & 0xF0u) | u);
-        else
-          *byte = (uint8_t)((*byte & 0x0Fu) | (uint8_t)(u << 4));
+        put_nibble(codes + n * (K / 2), k0 + k, (uint8_t)(q - qmin));
       }
     }
   }
+  free(grp);
   return status;
 }
 
@@ -629,4 +649,139 @@ int oracle_gemm_fp8(const uint8_t *qx, const float *sx, const uint8_t *qw,
     }
   }
   return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* GPTQ                                                                       */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * [P4] sec. 4.3: GPTQ quantizes a layer's weight column by column (input
+ * dimension by input dimension) and pushes each column's rounding error onto
+ * the columns not yet quantized, weighted by the inverse Hessian of the
+ * layer's reconstruction error ||X W^T - X W_hat^T||^2, H = 2 X^T X.  The
+ * page's skeleton uses the upper Cholesky factor U of H^-1 (damped by
+ * 0.01 * mean(diag(H)) so that H stays invertible): err = (w_i - q_i) / U_ii,
+ * W[:, i+1:] -= err * U[i, i+1:]; group parameters are recomputed at every
+ * group start from the current (corrected) weights.
+ */
+
+/* in-place Cholesky A = L L^T (lower, row-major); 0 on success */
+static int chol_lower(double *A, int64_t n) {
+  for (int64_t j = 0; j < n; ++j) {
+    double d = A[j * n + j];
+    for (int64_t k = 0; k < j; ++k) d -= A[j * n + k] * A[j * n + k];
+    if (!(d > 0.0)) return -1;
+    const double ljj = sqrt(d);
+    A[j * n + j] = ljj;
+    for (int64_t i = j + 1; i < n; ++i) {
+      double v = A[i * n + j];
+      for (int64_t k = 0; k < j; ++k) v -= A[i * n + k] * A[j * n + k];
+      A[i * n + j] = v / ljj;
+    }
+    for (int64_t i = 0; i < j; ++i) A[i * n + j] = 0.0;  /* clear the upper part */
+  }
+  return 0;
+}
+
+int oracle_gptq_hinv_chol(const void *X, int x_dtype, int64_t T, int64_t K,
+                          double damp, double *U) {
+  if (T <= 0 || K <= 0 || damp < 0.0) return ORACLE_ERR_ARG;
+  double *H = (double *)calloc((size_t)(K * K), sizeof(double));
+  double *Hi = (double *)calloc((size_t)(K * K), sizeof(double));
+  if (!H || !Hi) { free(H); free(Hi); return ORACLE_ERR_ARG; }
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t a = 0; a < K; ++a) {
+      const double xa = load_elem(X, x_dtype, t * K + a);
+      for (int64_t b = 0; b < K; ++b) H[a * K + b] += 2.0 * xa * load_elem(X, x_dtype, t * K + b);
+    }
+  double mean = 0.0;
+  for (int64_t a = 0; a < K; ++a) mean += H[a * K + a];
+  mean /= (double)K;
+  for (int64_t a = 0; a < K; ++a) H[a * K + a] += damp * mean;
+  int st = ORACLE_OK;
+  if (chol_lower(H, K) != 0) { st = ORACLE_ERR_ARG; goto done; }
+  /* H^-1 = L^-T L^-1: solve L y = e_c, then L^T x = y for every column c */
+  {
+    double *col = (double *)malloc((size_t)K * sizeof(double));
+    if (!col) { st = ORACLE_ERR_ARG; goto done; }
+    for (int64_t c = 0; c < K; ++c) {
+      for (int64_t i = 0; i < K; ++i) {            /* forward: L y = e_c */
+        double v = (i == c) ? 1.0 : 0.0;
+        for (int64_t k = 0; k < i; ++k) v -= H[i * K + k] * col[k];
+        col[i] = v / H[i * K + i];
+      }
+      for (int64_t i = K - 1; i >= 0; --i) {       /* backward: L^T x = y */
+        double v = col[i];
+        for (int64_t k = i + 1; k < K; ++k) v -= H[k * K + i] * col[k];
+        col[i] = v / H[i * K + i];
+      }
+      for (int64_t i = 0; i < K; ++i) Hi[i * K + c] = col[i];
+    }
+    free(col);
+  }
+  if (chol_lower(Hi, K) != 0) { st = ORACLE_ERR_ARG; goto done; }
+  for (int64_t i = 0; i < K; ++i)                  /* U = L^T (upper) */
+    for (int64_t j = 0; j < K; ++j) U[i * K + j] = (j >= i) ? Hi[j * K + i] : 0.0;
+done:
+  free(H);
+  free(Hi);
+  return st;
+}
+
+int oracle_gptq_quantize(const void *W, int w_dtype, int64_t N, int64_t K,
+                         const double *U, int group_size, int sym,
+                         uint8_t *codes, uint16_t *scales, uint16_t *zeros) {
+  if (N < 0 || K <= 0 || group_size <= 0 || (K % group_size) != 0 || (K % 2) != 0)
+    return ORACLE_ERR_ARG;
+  if (!sym && zeros == NULL) return ORACLE_ERR_ARG;
+  const int64_t G = K / group_size;
+  const int qmin = sym ? -8 : 0, qmax = sym ? 7 : 15;
+  double *work = (double *)malloc((size_t)K * sizeof(double));
+  float *grp = (float *)malloc((size_t)group_size * sizeof(float));
+  if (!work || !grp) {
+    free(work);
+    free(grp);
+    return ORACLE_ERR_ARG;
+  }
+  int status = ORACLE_OK;
+  memset(codes, 0, (size_t)(N * (K / 2)));
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) work[k] = load_elem(W, w_dtype, n * K + k);
+    float sf = 1.0f;
+    int z = 0, degenerate = 1;
+    for (int64_t k = 0; k < K; ++k) {
+      if (k % group_size == 0) {
+        /* parameters of the group starting here, from the corrected weights
+         * (rounded to binary32, the precision the INT4 rules work in) */
+        const int64_t g = k / group_size;
+        for (int64_t j = 0; j < group_size; ++j) grp[j] = (float)work[k + j];
+        uint16_t s16;
+        int nonfinite = 0;
+        group_params(grp, group_size, sym, &s16, &z, &degenerate, &nonfinite);
+        if (nonfinite) status = ORACLE_ERR_NONFINITE;
+        scales[n * G + g] = s16;
+        if (!sym) zeros[n * G + g] = oracle_f32_to_f16((float)z);
+        sf = oracle_f16_to_f32(s16);
+        if (isinf(sf)) status = ORACLE_ERR_NONFINITE;
+      }
+      const double w = work[k];
+      int q = 0;
+      double w_hat = 0.0;
+      if (!degenerate) {
+        /* the INT4 rule on the binary32 value: one fp32 division, half to even */
+        float r = oracle_round_half_even((float)w / sf);
+        r = fmaxf(-64.0f, fminf(64.0f, r));
+        q = clamp_int((int)r + z, qmin, qmax);
+        w_hat = (double)sf * (double)(q - (sym ? 0 : z));
+      }
+      put_nibble(codes + n * (K / 2), k, (uint8_t)(q - qmin));
+      /* this column's error, pushed into the columns not yet quantized */
+      const double e = (w - w_hat) / U[k * K + k];
+      for (int64_t j = k + 1; j < K; ++j) work[j] -= e * U[k * K + j];
+    }
+  }
+  free(work);
+  free(grp);
+  return status;
 }

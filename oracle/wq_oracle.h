@@ -20,8 +20,8 @@
  *   [P4] "27届大模型面试准备（十九）：模型量化全攻略" sec. 2.1 (affine quantization,
  *        min-max scale), 2.2 (per-group g=128, 4.25-bit), 3 (per-tensor worked
  *        example), 2.3 (FP8 E4M3 as an 8-bit format), 4.2 (SmoothQuant
- *        smoothing), 6 (per-token absmax quantizer, KV-cache: K per channel,
- *        V per token)
+ *        smoothing), 4.3 (GPTQ), 6 (per-token absmax quantizer, KV-cache: K
+ *        per channel, V per token)
  *
  * Status codes returned by the oracle functions.
  */
@@ -131,6 +131,20 @@ int oracle_gemm_fp8(const uint8_t *qx, const float *sx, const uint8_t *qw,
                     const float *sw, int64_t M, int64_t N, int64_t K,
                     int64_t m0, int64_t m1, int64_t n0, int64_t n1, double *Y,
                     double *acc);
+
+/* GPTQ ([P4] sec. 4.3).  Hessian factor from calibration activations X [T, K]:
+ * H = 2 X^T X + damp * mean(diag(H)) * I, U = upper Cholesky factor of H^-1
+ * (H^-1 = U^T U), binary64 [K, K] row-major.  ORACLE_ERR_ARG if H is not
+ * positive definite. */
+int oracle_gptq_hinv_chol(const void *X, int x_dtype, int64_t T, int64_t K,
+                          double damp, double *U);
+/* GPTQ INT4 group-wise quantization of W [N, K] with factor U: columns in
+ * order, group parameters from the error-corrected weights at each group
+ * start (the rules of oracle_quantize_int4), each column's scaled error pushed
+ * into the later columns.  Output format as oracle_quantize_int4. */
+int oracle_gptq_quantize(const void *W, int w_dtype, int64_t N, int64_t K,
+                         const double *U, int group_size, int sym,
+                         uint8_t *codes, uint16_t *scales, uint16_t *zeros);
 
 /* W8A8 rescale in fp64: Y = acc * sx[m] * sw[n] over the same window. */
 int oracle_w8a8_rescale(const int32_t *acc, const float *sx, const float *sw,
