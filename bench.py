@@ -478,6 +478,29 @@ def secondary(wq, dev, args):
     del W8, X8, Y8, ws8, fw, fsw
     torch.cuda.empty_cache()
 
+    # GPTQ of a [4096, 4096] bf16 weight (the 7B square projection), factor
+    # from 8192 synthetic correlated calibration tokens (numpy, not timed)
+    K = 4096
+    rng = np.random.default_rng(12)
+    Xc = rng.standard_normal((8192, K // 8)) @ rng.standard_normal((K // 8, K))
+    Xc += 0.2 * rng.standard_normal((8192, K))
+    H = 2.0 * Xc.T @ Xc
+    H += 0.01 * np.mean(np.diag(H)) * np.eye(K)
+    Ucpu = np.linalg.cholesky(np.linalg.inv(H)).T.copy()   # upper, H^-1 = U^T U
+    del Xc, H
+    Ug = torch.from_numpy(Ucpu).to(dev)
+    Wg = WORKLOADS["7b-decode"].weight(0).to(dev)
+    ws_g = torch.empty((int(wq.lib().wq_gptq_workspace_bytes(K, K)),), dtype=torch.uint8,
+                       device=dev)
+    cg = torch.empty((K, K // 2), dtype=torch.uint8, device=dev)
+    sg = torch.empty((K, K // 128), dtype=torch.float16, device=dev)
+    t = time_flushed(lambda: wq.wq_gptq_quantize(Wg, Ug, 128, True, cg, sg, None, ws_g), flush,
+                     reps=3, warm=1)
+    out["gptq_4096x4096_ms"] = round(t, 3)
+    out["gptq_4096x4096_fp64_tflops"] = round(2.0 * K * K * K / 2 / (t * 1e-3) / 1e12, 2)
+    del Ug, Wg, ws_g, cg, sg
+    torch.cuda.empty_cache()
+
     # KV-cache INT8 (K per channel, V per token), bf16 cache of 8 kv heads x 8
     # sequences x 8192 tokens x 128 dims (2 x 134 MB, larger than L2).  The
     # algorithmic bytes count one read of K and V, the int8 writes and the

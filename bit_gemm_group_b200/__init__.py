@@ -41,6 +41,7 @@ EXPORTED = (
     "wq_gemm_w4a16_noalloc",
     "wq_channel_absmax", "wq_smooth_scales", "wq_quantize_i8_smooth", "wq_quant_act_i8_smooth",
     "wq_gemm_w8a8_smooth", "wq_quant_kv", "wq_quantize_fp8_rows", "wq_gemm_fp8",
+    "wq_gptq_workspace_bytes", "wq_gptq_quantize",
 )
 
 
@@ -109,10 +110,14 @@ def _declare(L):
     L.wq_quant_kv.argtypes = [_P, _P, _INT, _I64, _I64, _I64, _P, _P, _P, _P, _P]
     L.wq_quantize_fp8_rows.argtypes = [_P, _INT, _I64, _I64, _P, _P, _P]
     L.wq_gemm_fp8.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P, _P, _SZ, _P, _P]
+    L.wq_gptq_workspace_bytes.argtypes = [_I64, _I64]
+    L.wq_gptq_workspace_bytes.restype = _SZ
+    L.wq_gptq_quantize.argtypes = [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P, _P, _SZ, _P]
     for name in ("wq_quantize_pack", "wq_dequant", "wq_gemm_w4a16", "wq_quant_act_i8",
                  "wq_gemm_w8a8", "wq_get_device_status", "wq_channel_absmax",
                  "wq_smooth_scales", "wq_quantize_i8_smooth", "wq_quant_act_i8_smooth",
-                 "wq_gemm_w8a8_smooth", "wq_quant_kv", "wq_quantize_fp8_rows", "wq_gemm_fp8"):
+                 "wq_gemm_w8a8_smooth", "wq_quant_kv", "wq_quantize_fp8_rows", "wq_gemm_fp8",
+                 "wq_gptq_quantize"):
         getattr(L, name).restype = _INT
 
 
@@ -262,6 +267,14 @@ def wq_gemm_fp8(X, Wq, w_scales, Y, ws, acc_out=None, stream=None):
     st = lib().wq_gemm_fp8(_ptr(X), M, K, _ptr(Wq), _ptr(w_scales), N, _ptr(Y), _ptr(ws),
                            ws.numel() * ws.element_size(), _ptr(acc_out), _stream(stream))
     _check(st, "wq_gemm_fp8")
+
+
+def wq_gptq_quantize(W, U, group_size, sym, codes, scales, zeros, ws, stream=None):
+    N, K = W.shape
+    st = lib().wq_gptq_quantize(_ptr(W), _DTYPE_TAG.get(W.dtype, -1), N, K, _ptr(U), group_size,
+                                int(bool(sym)), _ptr(codes), _ptr(scales), _ptr(zeros),
+                                _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "wq_gptq_quantize")
 
 
 def wq_get_device_status(reset=True, stream=None):
@@ -418,3 +431,19 @@ def gemm_fp8(X, Wq, w_scales, want_acc=False):
     acc = torch.empty((M, N), dtype=torch.float32, device=X.device) if want_acc else None
     wq_gemm_fp8(X, Wq, w_scales, Y, ws, acc)
     return (Y, acc) if want_acc else Y
+
+
+# ------------------------------------------------------------------ GPTQ helper
+
+def gptq_quantize(W, U, sym=True, group_size=128):
+    """GPTQ INT4 of W [N, K] with the fp64 factor U [K, K] (device tensors):
+    (codes, scales, zeros) in the wq_quantize_pack format."""
+    N, K = W.shape
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N, K // group_size), dtype=torch.float16, device=W.device)
+    zeros = None if sym else torch.empty((N, K // group_size), dtype=torch.float16,
+                                         device=W.device)
+    ws = torch.empty((max(1, int(lib().wq_gptq_workspace_bytes(N, K))),), dtype=torch.uint8,
+                     device=W.device)
+    wq_gptq_quantize(W, U, group_size, sym, codes, scales, zeros, ws)
+    return codes, scales, zeros

@@ -21,6 +21,9 @@ int launch_quant_kv(const void* Kc, const void* Vc, int dtype, int64_t BH, int64
                     void* qk, void* sk, void* qv, void* sv, cudaStream_t s);
 int launch_quantize_rows_fp8(const void* W, int w_dtype, int64_t R, int64_t K, void* q,
                              void* scales, cudaStream_t s);
+size_t gptq_workspace_bytes(int64_t N, int64_t K);
+int launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const double* U, int sym,
+                void* codes, void* scales, void* zeros, void* ws, cudaStream_t s);
 int launch_gemm_fp8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
                     int64_t N, void* Y, void* ws, void* acc_out, cudaStream_t s);
 int launch_dequant_int4(const void* codes, const void* scales, const void* zeros, int64_t N,

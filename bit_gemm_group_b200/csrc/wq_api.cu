@@ -351,6 +351,35 @@ int wq_gemm_fp8(const void* X, int64_t M, int64_t K, const void* Wq, const void*
   return wq_host::launch_gemm_fp8(X, M, K, Wq, w_scales, N, Y, ws, acc_out, as_stream(stream));
 }
 
+// -------------------------------------------------------------------- GPTQ
+
+size_t wq_gptq_workspace_bytes(int64_t N, int64_t K) {
+  if (N <= 0 || K <= 0) return 0;
+  return wq_host::gptq_workspace_bytes(N, K);
+}
+
+int wq_gptq_quantize(const void* W, int w_dtype, int64_t N, int64_t K, const void* U,
+                     int group_size, int sym, void* codes, void* scales, void* zeros, void* ws,
+                     size_t ws_bytes, void* stream) {
+  if (N < 0 || K < 0) return WQ_ERR_ARG;
+  if (w_dtype != WQ_F32 && w_dtype != WQ_BF16 && w_dtype != WQ_F16) return WQ_ERR_ARG;
+  if (sym != 0 && sym != 1) return WQ_ERR_ARG;
+  if ((sym == 1) != (zeros == nullptr)) return WQ_ERR_ARG;
+  if (group_size != 128) return WQ_ERR_UNSUPPORTED;
+  if ((K % 128) != 0) return WQ_ERR_ALIGN;
+  if (N > (int64_t(1) << 30) || K > (int64_t(1) << 20)) return WQ_ERR_UNSUPPORTED;
+  if (N == 0 || K == 0) return WQ_OK;
+  if (!W || !U || !codes || !scales) return WQ_ERR_ARG;
+  if (!ws || ws_bytes < wq_host::gptq_workspace_bytes(N, K)) return WQ_ERR_WORKSPACE;
+  if (!aligned16(W) || !aligned16(U) || !aligned16(codes) || !aligned16(scales) ||
+      (zeros && !aligned16(zeros)) || !aligned16(ws))
+    return WQ_ERR_ALIGN;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  return wq_host::launch_gptq(W, w_dtype, N, K, static_cast<const double*>(U), sym, codes,
+                              scales, zeros, ws, as_stream(stream));
+}
+
 int wq_get_device_status(void* stream, int reset) {
   int st = wq_host::ensure_device();
   if (st != WQ_OK) return st;

@@ -289,6 +289,27 @@ WQ_API int wq_gemm_fp8(const void *X, int64_t M, int64_t K, const void *Wq,
                        size_t ws_bytes, void *acc_out, void *stream);
 
 /*
+ * wq_gptq_quantize -- GPTQ INT4 group-wise quantization with error feedback
+ * ([P4] sec. 4.3).  Columns (input dims) are quantized in order; each column's
+ * error (w - w_hat) / U[i, i] is pushed into the columns not yet quantized
+ * with weights U[i, j]; at every group start the group's scale (and zero
+ * point) come from the corrected weights by the rules of wq_quantize_pack.
+ * U: fp64 [K, K] row-major, the upper Cholesky factor of the damped inverse
+ * Hessian, H^-1 = U^T U with H = 2 X^T X + damp * mean(diag(H)) * I from
+ * calibration activations X (damp 0.01 in [P4]); computing it is the
+ * caller's (it is a per-layer calibration step).  W [N, K] of w_dtype;
+ * outputs as wq_quantize_pack (bits 4, group_size 128 only).  The
+ * corrections run in binary64 and the rounding decision in binary32.
+ * ws: wq_gptq_workspace_bytes(N, K) bytes (fp64 errors), any contents.
+ * Requires K % 128 == 0.
+ */
+WQ_API size_t wq_gptq_workspace_bytes(int64_t N, int64_t K);
+WQ_API int wq_gptq_quantize(const void *W, int w_dtype, int64_t N, int64_t K,
+                            const void *U, int group_size, int sym, void *codes,
+                            void *scales, void *zeros, void *ws, size_t ws_bytes,
+                            void *stream);
+
+/*
  * wq_get_device_status -- synchronize `stream`, then return the first error
  * any kernel recorded since the last reset (WQ_OK if none); clear it when
  * reset != 0.  Returns WQ_ERR_CUDA if the synchronization itself fails.

@@ -135,3 +135,13 @@ def test_fp8_validation(L):
     assert L.wq_gemm_fp8(FAKE, 8, 128, FAKE, FAKE, 24, FAKE, FAKE, 1 << 20, None, None) == wq.WQ_ERR_ALIGN
     assert L.wq_gemm_fp8(FAKE, 8, 128, FAKE, FAKE, 16, FAKE, FAKE, 0, None, None) == wq.WQ_ERR_WORKSPACE
     assert L.wq_gemm_fp8(FAKE, 8, 128, None, FAKE, 16, FAKE, FAKE, 1 << 20, None, None) == wq.WQ_ERR_ARG
+
+
+def test_gptq_validation(L):
+    q = L.wq_gptq_quantize
+    assert q(FAKE, 1, 8, 256, FAKE, 64, 1, FAKE, FAKE, None, FAKE, 1 << 20, None) == wq.WQ_ERR_UNSUPPORTED
+    assert q(FAKE, 1, 8, 200, FAKE, 128, 1, FAKE, FAKE, None, FAKE, 1 << 20, None) == wq.WQ_ERR_ALIGN
+    assert q(FAKE, 1, 8, 256, FAKE, 128, 0, FAKE, FAKE, None, FAKE, 1 << 20, None) == wq.WQ_ERR_ARG
+    assert q(FAKE, 1, 8, 256, FAKE, 128, 1, FAKE, FAKE, None, FAKE, 16, None) == wq.WQ_ERR_WORKSPACE
+    assert q(FAKE, 1, 8, 256, None, 128, 1, FAKE, FAKE, None, FAKE, 1 << 20, None) == wq.WQ_ERR_ARG
+    assert L.wq_gptq_workspace_bytes(8, 256) == 8 * 256 * 8
