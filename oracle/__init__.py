@@ -74,6 +74,7 @@ def _declare(L):
     L.oracle_quantize_fp8_rows.argtypes = [_P, _INT, _I64, _I64, _P, _P]
     L.oracle_gemm_fp8.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _I64,
                                   _P, _P]
+    L.oracle_gemm_w8a16.argtypes = [_P, _I64, _I64, _P, _INT, _P, _I64, _I64, _I64, _P]
     L.oracle_gptq_hinv_chol.argtypes = [_P, _INT, _I64, _I64, ctypes.c_double, _P]
     L.oracle_gptq_quantize.argtypes = [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P]
     for name in ("oracle_quantize_int4", "oracle_quantize_int8_rows",
@@ -83,7 +84,7 @@ def _declare(L):
                  "oracle_channel_absmax", "oracle_smooth_scales",
                  "oracle_quantize_int8_rows_smoothed", "oracle_quant_act_i8_smoothed",
                  "oracle_quant_kv", "oracle_quantize_fp8_rows", "oracle_gemm_fp8",
-                 "oracle_gptq_hinv_chol", "oracle_gptq_quantize"):
+                 "oracle_gemm_w8a16", "oracle_gptq_hinv_chol", "oracle_gptq_quantize"):
         getattr(L, name).restype = _INT
 
 
@@ -266,6 +267,24 @@ def gemm_fp8(qx, sx, qw, sw, m0, m1, n0, n1):
     st = lib().oracle_gemm_fp8(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), M, N, K, m0, m1, n0, n1,
                                _ptr(Y), _ptr(acc))
     return Y, acc, st
+
+
+W_I8, W_E4M3 = 0, 1
+
+
+def gemm_w8a16(X_bf16_bits, qw, w_fmt, sw, n0=0, n1=None):
+    """fp64 Y[:, n0:n1] = X * (diag(sw) value(qw))^T, 8-bit weights (int8
+    codes or E4M3 bytes), X as uint16 bf16 bits [M, K]: (Y, status)."""
+    X = _c(X_bf16_bits, np.uint16)
+    qw = _c(qw.view(np.uint8) if qw.dtype == np.int8 else qw, np.uint8)
+    sw = _c(sw, np.float32)
+    M, K = X.shape
+    N = qw.shape[0]
+    n1 = N if n1 is None else n1
+    Y = np.zeros((M, n1 - n0), np.float64)
+    st = lib().oracle_gemm_w8a16(_ptr(X), M, K, _ptr(qw), int(w_fmt), _ptr(sw), N, n0, n1,
+                                 _ptr(Y))
+    return Y, st
 
 
 def gptq_hinv_chol(X, damp=0.01, dtype_tag=None):

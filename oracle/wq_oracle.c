@@ -651,6 +651,31 @@ int oracle_gemm_fp8(const uint8_t *qx, const float *sx, const uint8_t *qw,
   return ORACLE_OK;
 }
 
+/* [P4] sec. 2.3: W8A16 keeps the activations in 16 bits and expands the
+ * 8-bit weight before the product; with a per-output-channel scale the
+ * expanded weight is s[n] times the code's value. */
+int oracle_gemm_w8a16(const uint16_t *X, int64_t M, int64_t K, const uint8_t *qw,
+                      int w_fmt, const float *sw, int64_t N, int64_t n0, int64_t n1,
+                      double *Y) {
+  if (n0 < 0 || n1 > N || n0 > n1 || K <= 0 || M < 0) return ORACLE_ERR_ARG;
+  if (w_fmt != ORACLE_W_I8 && w_fmt != ORACLE_W_E4M3) return ORACLE_ERR_ARG;
+  const int64_t W = n1 - n0;
+  for (int64_t n = n0; n < n1; ++n) {
+    for (int64_t m = 0; m < M; ++m) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        const uint8_t c = qw[n * K + k];
+        const double v = (w_fmt == ORACLE_W_I8) ? (double)(int8_t)c
+                                                : (double)oracle_e4m3_to_f32(c);
+        const double w = (double)sw[n] * v;
+        acc += (double)oracle_bf16_to_f32(X[m * K + k]) * w;
+      }
+      Y[m * W + (n - n0)] = acc;
+    }
+  }
+  return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------------------- */
 /* GPTQ                                                                       */
 /* ------------------------------------------------------------------------- */

@@ -132,6 +132,17 @@ int oracle_gemm_fp8(const uint8_t *qx, const float *sx, const uint8_t *qw,
                     int64_t m0, int64_t m1, int64_t n0, int64_t n1, double *Y,
                     double *acc);
 
+/* W8A16 ([P4] sec. 2.3 naming table: 8-bit weights, 16-bit activations;
+ * the weight is expanded to the activation type inside the product).
+ * Weights are per-output-channel: x_hat[n, k] = sw[n] * value(qw[n, k]),
+ * value = the int8 code (w_fmt ORACLE_W_I8) or the E4M3 value
+ * (ORACLE_W_E4M3).  Y[m, n - n0] = sum_k X[m, k] * x_hat[n, k] in binary64
+ * for n in [n0, n1); X bf16 bits [M, K]; Y [M, n1 - n0]. */
+enum { ORACLE_W_I8 = 0, ORACLE_W_E4M3 = 1 };
+int oracle_gemm_w8a16(const uint16_t *X, int64_t M, int64_t K, const uint8_t *qw,
+                      int w_fmt, const float *sw, int64_t N, int64_t n0, int64_t n1,
+                      double *Y);
+
 /* GPTQ ([P4] sec. 4.3).  Hessian factor from calibration activations X [T, K]:
  * H = 2 X^T X + damp * mean(diag(H)) * I, U = upper Cholesky factor of H^-1
  * (H^-1 = U^T U), binary64 [K, K] row-major.  ORACLE_ERR_ARG if H is not
