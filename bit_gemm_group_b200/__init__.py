@@ -41,7 +41,7 @@ EXPORTED = (
     "wq_gemm_w4a16_noalloc",
     "wq_channel_absmax", "wq_smooth_scales", "wq_quantize_i8_smooth", "wq_quant_act_i8_smooth",
     "wq_gemm_w8a8_smooth", "wq_quant_kv", "wq_quantize_fp8_rows", "wq_gemm_fp8",
-    "wq_gptq_workspace_bytes", "wq_gptq_quantize",
+    "wq_gptq_workspace_bytes", "wq_gptq_quantize", "wq_gemm_w8a16",
 )
 
 
@@ -110,6 +110,7 @@ def _declare(L):
     L.wq_quant_kv.argtypes = [_P, _P, _INT, _I64, _I64, _I64, _P, _P, _P, _P, _P]
     L.wq_quantize_fp8_rows.argtypes = [_P, _INT, _I64, _I64, _P, _P, _P]
     L.wq_gemm_fp8.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P, _P, _SZ, _P, _P]
+    L.wq_gemm_w8a16.argtypes = [_P, _I64, _I64, _P, _INT, _P, _I64, _P, _P]
     L.wq_gptq_workspace_bytes.argtypes = [_I64, _I64]
     L.wq_gptq_workspace_bytes.restype = _SZ
     L.wq_gptq_quantize.argtypes = [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P, _P, _SZ, _P]
@@ -142,6 +143,13 @@ def _ptr(t):
     if not t.is_contiguous():
         raise WQError(WQ_ERR_ARG, "tensor must be contiguous (row-major)")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _bf16(t, what):
+    """Pointer of a tensor that an entry point takes as bf16 (no dtype tag)."""
+    if isinstance(t, torch.Tensor) and t.dtype != torch.bfloat16:
+        raise WQError(WQ_ERR_ARG, f"{what} must be bfloat16, got {t.dtype}")
+    return _ptr(t)
 
 
 def _stream(stream):
@@ -177,8 +185,8 @@ def wq_w4a16_workspace_bytes(M, N, K):
 def wq_gemm_w4a16(X, codes, scales, zeros, N, group_size, sym, Y, ws=None, stream=None):
     M, K = X.shape
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
-    st = lib().wq_gemm_w4a16(_ptr(X), M, K, _ptr(codes), _ptr(scales), _ptr(zeros), N,
-                             group_size, int(bool(sym)), _ptr(Y), _ptr(ws), ws_bytes,
+    st = lib().wq_gemm_w4a16(_bf16(X, "X"), M, K, _ptr(codes), _ptr(scales), _ptr(zeros), N,
+                             group_size, int(bool(sym)), _bf16(Y, "Y"), _ptr(ws), ws_bytes,
                              _stream(stream))
     _check(st, "wq_gemm_w4a16")
 
@@ -188,14 +196,15 @@ def wq_gemm_w4a16_noalloc(X, codes, scales, zeros, N, group_size, sym, Y, stream
     allocation.  Overlapping calls race; the first call per device must not
     be inside a stream capture."""
     M, K = X.shape
-    st = lib().wq_gemm_w4a16_noalloc(_ptr(X), M, K, _ptr(codes), _ptr(scales), _ptr(zeros), N,
-                                     group_size, int(bool(sym)), _ptr(Y), _stream(stream))
+    st = lib().wq_gemm_w4a16_noalloc(_bf16(X, "X"), M, K, _ptr(codes), _ptr(scales),
+                                     _ptr(zeros), N, group_size, int(bool(sym)), _bf16(Y, "Y"),
+                                     _stream(stream))
     _check(st, "wq_gemm_w4a16_noalloc")
 
 
 def wq_quant_act_i8(X, q, s, stream=None):
     M, K = X.shape
-    st = lib().wq_quant_act_i8(_ptr(X), M, K, _ptr(q), _ptr(s), _stream(stream))
+    st = lib().wq_quant_act_i8(_bf16(X, "X"), M, K, _ptr(q), _ptr(s), _stream(stream))
     _check(st, "wq_quant_act_i8")
 
 
@@ -206,8 +215,9 @@ def wq_w8a8_workspace_bytes(M, K):
 def wq_gemm_w8a8(X, Wq, w_scales, Y, ws, acc_out=None, stream=None):
     M, K = X.shape
     N = Wq.shape[0]
-    st = lib().wq_gemm_w8a8(_ptr(X), M, K, _ptr(Wq), _ptr(w_scales), N, _ptr(Y), _ptr(ws),
-                            ws.numel() * ws.element_size(), _ptr(acc_out), _stream(stream))
+    st = lib().wq_gemm_w8a8(_bf16(X, "X"), M, K, _ptr(Wq), _ptr(w_scales), N, _bf16(Y, "Y"),
+                            _ptr(ws), ws.numel() * ws.element_size(), _ptr(acc_out),
+                            _stream(stream))
     _check(st, "wq_gemm_w8a8")
 
 
@@ -233,7 +243,7 @@ def wq_quantize_i8_smooth(W, s, q, scales, stream=None):
 
 def wq_quant_act_i8_smooth(X, s, q, sx, stream=None):
     M, K = X.shape
-    st = lib().wq_quant_act_i8_smooth(_ptr(X), M, K, _ptr(s), _ptr(q), _ptr(sx),
+    st = lib().wq_quant_act_i8_smooth(_bf16(X, "X"), M, K, _ptr(s), _ptr(q), _ptr(sx),
                                       _stream(stream))
     _check(st, "wq_quant_act_i8_smooth")
 
@@ -241,9 +251,9 @@ def wq_quant_act_i8_smooth(X, s, q, sx, stream=None):
 def wq_gemm_w8a8_smooth(X, Wq, w_scales, s, Y, ws, acc_out=None, stream=None):
     M, K = X.shape
     N = Wq.shape[0]
-    st = lib().wq_gemm_w8a8_smooth(_ptr(X), M, K, _ptr(Wq), _ptr(w_scales), _ptr(s), N, _ptr(Y),
-                                   _ptr(ws), ws.numel() * ws.element_size(), _ptr(acc_out),
-                                   _stream(stream))
+    st = lib().wq_gemm_w8a8_smooth(_bf16(X, "X"), M, K, _ptr(Wq), _ptr(w_scales), _ptr(s), N,
+                                   _bf16(Y, "Y"), _ptr(ws), ws.numel() * ws.element_size(),
+                                   _ptr(acc_out), _stream(stream))
     _check(st, "wq_gemm_w8a8_smooth")
 
 
@@ -264,9 +274,21 @@ def wq_quantize_fp8_rows(A, q, scales, stream=None):
 def wq_gemm_fp8(X, Wq, w_scales, Y, ws, acc_out=None, stream=None):
     M, K = X.shape
     N = Wq.shape[0]
-    st = lib().wq_gemm_fp8(_ptr(X), M, K, _ptr(Wq), _ptr(w_scales), N, _ptr(Y), _ptr(ws),
-                           ws.numel() * ws.element_size(), _ptr(acc_out), _stream(stream))
+    st = lib().wq_gemm_fp8(_bf16(X, "X"), M, K, _ptr(Wq), _ptr(w_scales), N, _bf16(Y, "Y"),
+                           _ptr(ws), ws.numel() * ws.element_size(), _ptr(acc_out),
+                           _stream(stream))
     _check(st, "wq_gemm_fp8")
+
+
+WQ_W8_INT8, WQ_W8_E4M3 = 0, 1
+
+
+def wq_gemm_w8a16(X, Wq, w_fmt, w_scales, Y, stream=None):
+    M, K = X.shape
+    N = Wq.shape[0]
+    st = lib().wq_gemm_w8a16(_bf16(X, "X"), M, K, _ptr(Wq), int(w_fmt), _ptr(w_scales), N,
+                             _bf16(Y, "Y"), _stream(stream))
+    _check(st, "wq_gemm_w8a16")
 
 
 def wq_gptq_quantize(W, U, group_size, sym, codes, scales, zeros, ws, stream=None):
@@ -434,6 +456,17 @@ def gemm_fp8(X, Wq, w_scales, want_acc=False):
 
 
 # ------------------------------------------------------------------ GPTQ helper
+
+def gemm_w8a16(X, Wq, w_scales, w_fmt=None):
+    """W8A16 product of bf16 X [M, K] with 8-bit per-channel weights: int8
+    codes (from quantize_pack(W, K, 8)) or E4M3 codes (from
+    quantize_fp8_rows(W)); the format follows Wq's dtype unless given."""
+    if w_fmt is None:
+        w_fmt = WQ_W8_INT8 if Wq.dtype == torch.int8 else WQ_W8_E4M3
+    Y = torch.empty((X.shape[0], Wq.shape[0]), dtype=torch.bfloat16, device=X.device)
+    wq_gemm_w8a16(X, Wq, w_fmt, w_scales, Y)
+    return Y
+
 
 def gptq_quantize(W, U, sym=True, group_size=128):
     """GPTQ INT4 of W [N, K] with the fp64 factor U [K, K] (device tensors):

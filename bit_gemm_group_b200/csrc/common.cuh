@@ -24,8 +24,10 @@ __device__ __forceinline__ void record_error(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
-// One IEEE-754 binary32 division, round to nearest even (never a
-// reciprocal-multiply): the quantizer's codes depend on it bit for bit.
+// One IEEE-754 binary32 division, round to nearest even.  The quantizers'
+// codes are defined by this quotient bit for bit; their reciprocal-multiply
+// fast paths reproduce it exactly and fall back to it near rounding
+// boundaries.
 __device__ __forceinline__ float div_rn(float a, float b) { return __fdiv_rn(a, b); }
 
 // Round half to even on a float (numpy/torch `round` semantics).

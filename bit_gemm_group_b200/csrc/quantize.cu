@@ -7,7 +7,10 @@
 //
 // All of them stream their input once with 16-byte (or element-sized when
 // smaller) vector loads, keep several groups in flight per warp, and size the
-// grid as a multiple of the SM count.
+// grid as a multiple of the SM count.  The per-element IEEE division of the
+// codes is replaced by a reciprocal multiply whose rounding decisions are
+// proved equal (INT4 for 16-bit inputs; INT8 and E4M3 for every input type;
+// see the section below).
 #include "common.cuh"
 #include "kernels.h"
 #include <cuda_fp8.h>
@@ -147,6 +150,216 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// Reciprocal-multiply quantization with the IEEE-division result
+// ---------------------------------------------------------------------------
+// The quantizers' codes are defined by round-half-even of the binary32
+// quotient fl(x / s).  One reciprocal per scale and one multiply per element
+// reach the same codes: r = x * rcp(s), with rcp within one ulp of 1/s, is
+// within |x/s| * 1.5 * 2^-23 of x/s, and rint(fl(x/s)) depends only on which
+// side of each half-integer x/s lies.  So rint(r) is the IEEE result unless
+// x/s is very close to (or exactly on) a half-integer; each kernel below
+// recognises those elements and decides them exactly.
+
+// 1/v within one ulp (a single instruction).
+__device__ __forceinline__ float rcp_approx(float v) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// The two 16-bit floats of a 32-bit word as fp32 (element 0 = low half).
+template <typename T>
+__device__ __forceinline__ void unpack2(uint32_t w, float& a, float& b);
+template <>
+__device__ __forceinline__ void unpack2<__nv_bfloat16>(uint32_t w, float& a, float& b) {
+  a = __uint_as_float(w << 16);
+  b = __uint_as_float(w & 0xFFFF0000u);
+}
+template <>
+__device__ __forceinline__ void unpack2<__half>(uint32_t w, float& a, float& b) {
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+  a = f.x;
+  b = f.y;
+}
+
+// acc' = w * 0 + acc on the two 16-bit lanes: stays (+-)0 while every element
+// seen is finite and turns NaN, for good, at the first Inf or NaN.
+template <typename T>
+__device__ __forceinline__ uint32_t nonfinite_acc(uint32_t acc, uint32_t w);
+template <>
+__device__ __forceinline__ uint32_t nonfinite_acc<__nv_bfloat16>(uint32_t acc, uint32_t w) {
+  __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&acc);
+  a = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&w), __float2bfloat162_rn(0.f), a);
+  return *reinterpret_cast<const uint32_t*>(&a);
+}
+template <>
+__device__ __forceinline__ uint32_t nonfinite_acc<__half>(uint32_t acc, uint32_t w) {
+  __half2 a = *reinterpret_cast<const __half2*>(&acc);
+  a = __hfma2(*reinterpret_cast<const __half2*>(&w), __float2half2_rn(0.f), a);
+  return *reinterpret_cast<const uint32_t*>(&a);
+}
+__device__ __forceinline__ bool is_nonfinite_acc(uint32_t acc) { return (acc & 0x7FFF7FFFu) != 0; }
+
+// rint(fl(x / s)) for an INT8 code, from inv = rcp_approx(s).  Exact for
+// |x/s| <= 128.5: r = x * inv is within 2^-15.4 of x/s and fl(x/s) within
+// 2^-17, so rint(r) is the IEEE result unless r is within 2^-14 of a
+// half-integer, where the division itself decides.  Larger quotients
+// saturate the code either way.
+__device__ __forceinline__ float rint_quot_i8(float x, float s, float inv) {
+  const float r = x * inv;
+  const float k = rintf(r);
+  if (fabsf(fabsf(r - k) - 0.5f) <= 0x1p-14f) return rintf(div_rn(x, s));
+  return k;
+}
+
+// A binary32 quotient that rounds to the same E4M3 code as fl(x / s), from
+// inv = rcp_approx(s).  r = x * inv is within 3 units of the binary32 last
+// place of x/s, and fl(x/s) within half a unit; an E4M3 half-way point in the
+// normal range has the low 20 mantissa bits 0x80000 (bit 19 alone), so when
+// r's low 20 bits are more than 4 units from that pattern, r and fl(x/s) lie
+// on the same side of every half-way point and round to the same code
+// (powers of two, where the binade changes, are codes themselves).  Nonzero
+// |r| < 2^-6 (the E4M3 subnormal range, uniform spacing 2^-9) and the rare
+// near-half-way r take the division itself.
+__device__ __forceinline__ float quot_e4m3(float x, float s, float inv) {
+  const float r = x * inv;
+  const int m20 = int(__float_as_uint(r) & 0xFFFFFu) - 0x80000;
+  if ((r != 0.f && fabsf(r) < 0x1p-6f) || (m20 >= -4 && m20 <= 4)) return div_rn(x, s);
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// INT4 group-wise quantize + pack of 16-bit weights (bf16 / fp16), g <= 512
+// ---------------------------------------------------------------------------
+// Codes, scales and zeros equal quantize_int4_kernel's bit for bit.  Lane l
+// of a group's LPG lanes owns its 16 elements [16 l, 16 l + 16) (two 16-byte
+// loads, one 8-byte store of codes); a warp takes 32 / LPG adjacent groups per
+// step and U steps are loaded before any is processed.
+//
+// Exactness of the reciprocal multiply here: x is a 16-bit float and s an
+// fp16 scale, x = mx 2^a and s = ms 2^b with integer significands below 2^11.
+// Then x/s - (j + 1/2) is a multiple of 2^min(a - b, -1) / ms, so x/s is
+// either exactly a half-integer or more than 2^-14 away from every one (the
+// bound holds for every 16-bit x against every finite fp16 s; codes only
+// depend on |x/s| <= 24, beyond which the clamp saturates them either way,
+// and there r is within 2^-17.4 of x/s).  rint(r) is therefore exact except
+// at exact half-integers, which are recognised without rounding: with
+// k = rint(r), e = x - k s is exact in one fma (x and k s are within a factor
+// of two, or k = 0), and x/s is a half-integer iff |e| = s/2; the IEEE result
+// is then the even one of k and k + sign(e).
+template <typename T, int LPG, int U>
+__global__ void __launch_bounds__(256) quantize_int4_x16_kernel(
+    const T* __restrict__ W, int64_t total_groups, int sym, uint8_t* __restrict__ codes,
+    __half* __restrict__ scales, __half* __restrict__ zeros, int* status) {
+  constexpr int GS = 16 * LPG;   // group size
+  constexpr int GPW = 32 / LPG;  // groups per warp and step
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPG, li = lane % LPG;
+  const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  const int qmin = sym ? -8 : 0;
+  uint32_t nf = 0;
+  bool inf_scale = false;
+
+  for (int64_t base = warp * (U * GPW); base < total_groups; base += nwarps * (U * GPW)) {
+    uint4 in[U][2];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int64_t gi = base + j * GPW + sub;
+      if (gi < total_groups) {
+        const uint4* src = reinterpret_cast<const uint4*>(W + gi * GS) + 2 * li;
+        in[j][0] = __ldcs(src);
+        in[j][1] = __ldcs(src + 1);
+      } else {
+        in[j][0] = in[j][1] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      if (base + j * GPW >= total_groups) break;  // warp-uniform
+      const int64_t gi = base + j * GPW + sub;
+      const bool live = gi < total_groups;
+      const uint32_t w[8] = {in[j][0].x, in[j][0].y, in[j][0].z, in[j][0].w,
+                             in[j][1].x, in[j][1].y, in[j][1].z, in[j][1].w};
+      float x[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        unpack2<T>(w[i], x[2 * i], x[2 * i + 1]);
+        nf = nonfinite_acc<T>(nf, w[i]);
+      }
+      unsigned short s_bits;
+      float sf;
+      int z = 0;
+      bool degenerate;
+      if (sym) {
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(x[e]));
+#pragma unroll
+        for (int o = LPG / 2; o > 0; o >>= 1)
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        sf = f16_round_trip(div_rn(amax, 7.f), &s_bits);
+        degenerate = (amax < 1e-8f) || (sf == 0.f);
+        if (degenerate) sf = f16_round_trip(amax, &s_bits);
+      } else {
+        float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          mn = fminf(mn, x[e]);
+          mx = fmaxf(mx, x[e]);
+        }
+#pragma unroll
+        for (int o = LPG / 2; o > 0; o >>= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        const float range = mx - mn;
+        sf = f16_round_trip(div_rn(range, 15.f), &s_bits);
+        degenerate = (range < 1e-8f) || (sf == 0.f);
+        if (degenerate) {
+          sf = f16_round_trip(1.f, &s_bits);
+        } else {
+          const float zr = round_even(div_rn(-mn, sf));
+          z = int(fmaxf(0.f, fminf(15.f, zr)));
+        }
+      }
+      if (live && li == 0) {
+        scales[gi] = __ushort_as_half(s_bits);
+        if (!sym) zeros[gi] = __int2half_rn(z);
+      }
+      inf_scale |= isinf(sf);
+      const float inv = rcp_approx(sf), hs = 0.5f * sf;
+      float k[16];
+      bool tie = false;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        k[e] = rintf(x[e] * inv);
+        tie |= fabsf(fmaf(-k[e], sf, x[e])) == hs;
+      }
+      if (__any_sync(0xffffffffu, tie)) {  // exact half-way quotients: to even
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float d = fmaf(-k[e], sf, x[e]);
+          if (fabsf(d) == hs && (int(k[e]) & 1)) k[e] += copysignf(1.f, d);
+        }
+      }
+      const int zq = z - qmin;  // nibble = clamp(q + z, qmin, qmax) - qmin
+      uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int nib =
+            degenerate ? -qmin : min(max(__float2int_rn(fminf(k[e], 64.f)) + zq, 0), 15);
+        packed[e >> 3] |= uint32_t(nib) << (4 * (e & 7));
+      }
+      if (live)
+        *reinterpret_cast<uint2*>(codes + gi * (GS / 2) + li * 8) = make_uint2(packed[0], packed[1]);
+    }
+  }
+  if (__any_sync(0xffffffffu, is_nonfinite_acc(nf) || inf_scale) && lane == 0)
+    record_error(status, WQ_ERR_NONFINITE);
+}
+
+// ---------------------------------------------------------------------------
 // INT8 per-row quantization (weights per output channel / activations per token)
 // ---------------------------------------------------------------------------
 // One 256-thread block per row: pass 1 reduces amax with 16-byte loads, pass 2
@@ -215,6 +428,7 @@ __global__ void __launch_bounds__(256) quantize_rows_i8_kernel(
       if (bad_any) record_error(status, WQ_ERR_NONFINITE);
     }
     const int lo = ACT ? -128 : -127;
+    const float inv = rcp_approx(s);
     for (int64_t k = int64_t(threadIdx.x) * EV; k < K; k += int64_t(blockDim.x) * EV) {
       Elems<T, EV> v;
       v.load(row + k);
@@ -230,7 +444,7 @@ __global__ void __launch_bounds__(256) quantize_rows_i8_kernel(
       for (int e = 0; e < EV; ++e) {
         int qi = 0;
         if (!degenerate) {
-          float rr = round_even(div_rn(x[e], s));
+          float rr = rint_quot_i8(x[e], s, inv);
           rr = fmaxf(-200.f, fminf(200.f, rr));
           qi = min(max(int(rr), lo), 127);
         }
@@ -281,6 +495,7 @@ __global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(
     }
     __syncthreads();
     const float s = fmaxf(div_rn(red[0], 448.f), 1e-8f);
+    const float inv = rcp_approx(s);
     if (threadIdx.x == 0) {
       scales[r] = s;
       if (bad_any) record_error(status, WQ_ERR_NONFINITE);
@@ -294,8 +509,8 @@ __global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(
       } o;
 #pragma unroll
       for (int e = 0; e < EV; ++e)
-        o.b[e] = uint8_t(__nv_cvt_float_to_fp8(div_rn(to_f32<T>(v.u.e[e]), s), __NV_SATFINITE,
-                                               __NV_E4M3));
+        o.b[e] = uint8_t(__nv_cvt_float_to_fp8(quot_e4m3(to_f32<T>(v.u.e[e]), s, inv),
+                                               __NV_SATFINITE, __NV_E4M3));
       *reinterpret_cast<uint2*>(q + r * K + k) = o.v2;
     }
     __syncthreads();  // red[] is reused by the next row
@@ -432,13 +647,14 @@ __global__ void __launch_bounds__(256) kv_v_quant_kernel(const T* __restrict__ V
     for (int o = LPR / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float sc = fmaxf(div_rn(amax, 127.f), 1e-8f);
     if (act) {
+      const float inv = rcp_approx(sc);
       union {
         uint2 v2;
         int8_t b8[8];
       } o;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        float rr = round_even(div_rn(x[e], sc));
+        float rr = rint_quot_i8(x[e], sc, inv);
         rr = fmaxf(-200.f, fminf(200.f, rr));
         o.b8[e] = int8_t(min(max(int(rr), -128), 127));
       }
@@ -477,7 +693,7 @@ __global__ void __launch_bounds__(256) kv_k_quant_kernel(const T* __restrict__ K
     } o;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      float r = round_even(div_rn(to_f32<T>(v.u.e[e]), sc[e]));
+      float r = rint_quot_i8(to_f32<T>(v.u.e[e]), sc[e], rcp_approx(sc[e]));
       r = fmaxf(-200.f, fminf(200.f, r));
       o.b8[e] = int8_t(min(max(int(r), -128), 127));
     }
@@ -598,9 +814,35 @@ static void quantize_int4_typed(const void* W, int64_t N, int64_t K, int sym, vo
       static_cast<__half*>(scales), static_cast<__half*>(zeros), status_ptr());
 }
 
+// 16-bit weights, g = 16 LPG: the reciprocal-multiply kernel.
+template <typename T, int LPG>
+static void quantize_int4_x16(const void* W, int64_t N, int64_t K, int sym, void* codes,
+                              void* scales, void* zeros, cudaStream_t s) {
+  constexpr int U = 4;
+  const int64_t total = N * (K / (16 * LPG));
+  const int64_t steps = (total + U * (32 / LPG) - 1) / (U * (32 / LPG));  // warp steps
+  wq::quantize_int4_x16_kernel<T, LPG, U><<<grid_for(steps, 8), 256, 0, s>>>(
+      static_cast<const T*>(W), total, sym, static_cast<uint8_t*>(codes),
+      static_cast<__half*>(scales), static_cast<__half*>(zeros), status_ptr());
+}
+
 template <typename T>
 static int quantize_int4_dispatch(const void* W, int64_t N, int64_t K, int gs, int sym,
                                   void* codes, void* scales, void* zeros, cudaStream_t s) {
+  if constexpr (sizeof(T) == 2) {
+    if (gs <= 512) {
+      switch (gs) {
+        case 32: quantize_int4_x16<T, 2>(W, N, K, sym, codes, scales, zeros, s); break;
+        case 64: quantize_int4_x16<T, 4>(W, N, K, sym, codes, scales, zeros, s); break;
+        case 128: quantize_int4_x16<T, 8>(W, N, K, sym, codes, scales, zeros, s); break;
+        case 256: quantize_int4_x16<T, 16>(W, N, K, sym, codes, scales, zeros, s); break;
+        case 512: quantize_int4_x16<T, 32>(W, N, K, sym, codes, scales, zeros, s); break;
+        default: return WQ_ERR_UNSUPPORTED;
+      }
+      WQ_LAUNCH_CHECK("quantize_int4_x16_kernel");
+      return WQ_OK;
+    }
+  }
   switch (gs) {
     case 32: quantize_int4_typed<T, 1>(W, N, K, sym, codes, scales, zeros, s); break;
     case 64: quantize_int4_typed<T, 2>(W, N, K, sym, codes, scales, zeros, s); break;

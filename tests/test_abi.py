@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import bit_gemm_group_b200 as wq
 
@@ -145,3 +146,25 @@ def test_gptq_validation(L):
     assert q(FAKE, 1, 8, 256, FAKE, 128, 1, FAKE, FAKE, None, FAKE, 16, None) == wq.WQ_ERR_WORKSPACE
     assert q(FAKE, 1, 8, 256, None, 128, 1, FAKE, FAKE, None, FAKE, 1 << 20, None) == wq.WQ_ERR_ARG
     assert L.wq_gptq_workspace_bytes(8, 256) == 8 * 256 * 8
+
+
+def test_w8a16_validation(L):
+    assert L.wq_gemm_w8a16(FAKE, 2, 96, FAKE, 0, FAKE, 16, FAKE, None) == wq.WQ_ERR_ALIGN   # K % 64
+    assert L.wq_gemm_w8a16(FAKE, 2, 128, FAKE, 2, FAKE, 16, FAKE, None) == wq.WQ_ERR_ARG    # format
+    assert L.wq_gemm_w8a16(FAKE, 2, 128, None, 1, FAKE, 16, FAKE, None) == wq.WQ_ERR_ARG
+    assert L.wq_gemm_w8a16(FAKE, -1, 128, FAKE, 1, FAKE, 16, FAKE, None) == wq.WQ_ERR_ARG
+    assert L.wq_gemm_w8a16(MISALIGNED, 2, 128, FAKE, 0, FAKE, 16, FAKE, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_gemm_w8a16(FAKE, 0, 128, FAKE, 0, FAKE, 16, FAKE, None) == wq.WQ_OK
+
+
+def test_binding_rejects_non_bf16_activations():
+    """Entry points whose X and Y are bf16 by contract (no dtype argument)
+    refuse other dtypes in the binding, before any pointer is passed."""
+    X16 = torch.zeros((2, 16), dtype=torch.float16)
+    q = torch.zeros((2, 16), dtype=torch.int8)
+    s = torch.zeros((2,), dtype=torch.float32)
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_quant_act_i8(X16, q, s)
+    assert e.value.status == wq.WQ_ERR_ARG and "bfloat16" in str(e.value)
+    with pytest.raises(wq.WQError):
+        wq.wq_gemm_w4a16(X16, q, s, None, 8, 128, True, X16)

@@ -8,7 +8,7 @@ import torch
 import bit_gemm_group_b200 as wq
 import oracle
 from parity_util import oracle_input, u16
-from workloads import WORKLOADS, make_weight, make_activation
+from workloads import WORKLOADS, bf16_bits, make_weight, make_activation
 
 pytestmark = pytest.mark.gpu
 
@@ -167,3 +167,108 @@ def test_act_quant_ragged(M, K):
     X = make_activation(M, K, seed=M + K, outlier_dims=min(6, K // 8))
     X[0, :] = 0.0
     check_act(X)
+
+
+# ------------------------------------------- rounding boundaries of the codes
+# The quantizers reach fl(x / s) through a reciprocal multiply and decide
+# exact half-way quotients (and, for a binary32 scale, quotients within 2^-14
+# of a half-way point) separately.  These inputs put most elements on or next
+# to those boundaries; codes must still equal the oracle's IEEE-division ones.
+
+def _half_steps(n, step, lo, hi, seed):
+    """n values (j + 1/2) * step with integer j in [lo, hi), shuffled."""
+    g = torch.Generator().manual_seed(seed)
+    j = torch.randint(lo, hi, (n,), generator=g).double()
+    return ((j + 0.5) * step).float()
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("g", [32, 128, 512])
+def test_int4_half_way_quotients(dtype, g):
+    rows, K = 12, 2048
+    step = 0.0625  # the fp16 scale of every group: amax = 7 step, or range = 15 step
+    W = torch.empty(rows, K)
+    for r in range(rows):
+        W[r] = _half_steps(K, step, -7, 7, seed=r)
+    Ws, Wa = W.clone(), W.clone()
+    Ws.view(rows, K // g, g)[:, :, 0] = 7 * step          # sym: s = step
+    Wa.view(rows, K // g, g)[:, :, 0] = 7 * step
+    Wa.view(rows, K // g, g)[:, :, 1] = -8 * step         # asym: s = step, z = 8
+    Wa.view(rows, K // g, g)[1::2, :, 1] = -7 * step      # odd rows: range 14 step
+    check_int4(Ws.to(dtype), g, sym=True)
+    check_int4(Wa.to(dtype), g, sym=False)
+
+
+def _rows_with(X):
+    check_int8_rows(X)
+    if X.dtype != torch.bfloat16:  # the activation quantizer takes bf16 only
+        return
+    q, s = wq.quant_act_i8(X.cuda())
+    arr, tag = oracle_input(X)
+    oq, os_, st = oracle.quant_act_i8(arr, dtype_tag=tag)
+    np.testing.assert_array_equal(q.cpu().numpy(), oq)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("K", [64, 4096, 5120])
+def test_int8_rows_half_way(dtype, K):
+    """Row maximum 127 2^-7 (scale 2^-7 exactly), values on half-integer
+    multiples of the scale."""
+    R = 24
+    X = torch.stack([_half_steps(K, 2.0 ** -7, -127, 127, seed=r) for r in range(R)])
+    X[:, 0] = 127 * 2.0 ** -7
+    _rows_with(X.to(dtype))
+
+
+@pytest.mark.parametrize("K", [64, 4096])
+def test_int8_rows_close_to_half_way(K):
+    """fp16 rows (maximum 3) whose quotients by the binary32 scale 3/127 lie
+    within 2^-9 of a half-integer."""
+    s = np.float32(3.0) / np.float32(127.0)
+    vals = np.arange(1, 0x4200, dtype=np.uint16).view(np.float16).astype(np.float32)
+    vals = vals[vals < 3.0]
+    qv = vals / s
+    near = vals[np.abs(np.abs(qv - np.rint(qv)) - 0.5) < 2.0 ** -9]
+    assert near.size > 8
+    rng = np.random.default_rng(K)
+    X = rng.choice(near, size=(16, K)) * rng.choice([-1.0, 1.0], size=(16, K))
+    X[:, 0] = 3.0
+    _rows_with(torch.from_numpy(X.astype(np.float32)).to(torch.float16))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_fp8_rows_half_way(dtype):
+    """amax = 7 gives s = 2^-6; values on E4M3 half-way points (m + 1/2)
+    2^(e-3) times s, in the normal and subnormal E4M3 ranges."""
+    R, K = 16, 1024
+    rng = np.random.default_rng(3)
+    e = rng.integers(-9, 8, size=(R, K)).astype(np.float64)
+    m = rng.integers(8, 16, size=(R, K)).astype(np.float64)
+    v = (m + 0.5) * 2.0 ** (e - 3) * 2.0 ** -6 * rng.choice([-1.0, 1.0], size=(R, K))
+    v[:, 0] = 7.0
+    A = torch.from_numpy(v.astype(np.float32)).to(dtype)
+    q, s = wq.quantize_fp8_rows(A.cuda())
+    arr, tag = oracle_input(A)
+    oq, os_, st = oracle.quantize_fp8_rows(arr, dtype_tag=tag)
+    assert st == oracle.OK
+    np.testing.assert_array_equal(q.cpu().numpy(), oq)
+    np.testing.assert_array_equal(s.cpu().numpy(), os_)
+
+
+def test_kv_half_way():
+    """V rows and K channels whose scale is exactly 2^-7, values on
+    half-integer multiples of it."""
+    BH, S, D = 2, 64, 128
+    Kc = _half_steps(BH * S * D, 2.0 ** -7, -127, 127, seed=1).view(BH, S, D)
+    Vc = _half_steps(BH * S * D, 2.0 ** -7, -127, 127, seed=2).view(BH, S, D)
+    Kc[:, 0, :] = 127 * 2.0 ** -7
+    Vc[:, :, 0] = 127 * 2.0 ** -7
+    Kb, Vb = Kc.to(torch.bfloat16), Vc.to(torch.bfloat16)
+    qk, sk, qv, sv = wq.quant_kv(Kb.cuda(), Vb.cuda())
+    oqk, osk, oqv, osv, st = oracle.quant_kv(bf16_bits(Kb), bf16_bits(Vb), dtype_tag=oracle.BF16)
+    assert st == oracle.OK
+    np.testing.assert_array_equal(qk.cpu().numpy(), oqk)
+    np.testing.assert_array_equal(qv.cpu().numpy(), oqv)
+    np.testing.assert_array_equal(sk.cpu().numpy().view(np.uint32), osk.view(np.uint32))
+    np.testing.assert_array_equal(sv.cpu().numpy().view(np.uint32), osv.view(np.uint32))
