@@ -478,6 +478,30 @@ def secondary(wq, dev, args):
     del W8, X8, Y8, ws8, fw, fsw
     torch.cuda.empty_cache()
 
+    # W8A16 (int8 and E4M3 per-channel weights, bf16 activations): decode
+    # M = 1 on the 7B [11008, 4096] weight (HBM GB/s of codes + scales + X + Y)
+    # and prefill M = 2048 on the same weight (TFLOPS), L2 flushed between runs
+    W16 = WORKLOADS["7b-decode"].weight(1).to(dev)
+    N, K = W16.shape
+    Xd = WORKLOADS["7b-decode"].activation(1, K).to(dev)
+    Xp = WORKLOADS["prefill"].activation(2048, K).to(dev)
+    Yd = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+    Yp = torch.empty((2048, N), dtype=torch.bfloat16, device=dev)
+    for name, (q16, s16) in (("int8", wq.quantize_pack(W16, K, 8, True)[:2]),
+                             ("e4m3", wq.quantize_fp8_rows(W16))):
+        fmt = wq.WQ_W8_INT8 if name == "int8" else wq.WQ_W8_E4M3
+        t = time_flushed(lambda: wq.wq_gemm_w8a16(Xd, q16, fmt, s16, Yd), flush)
+        b = N * K + 4 * N + 2 * K + 2 * N
+        out[f"w8a16_{name}_decode_gbs"] = round(b / (t * 1e-3) / 1e9, 1)
+        out[f"w8a16_{name}_decode_frac_hbm"] = round(b / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 3)
+        t = time_flushed(lambda: wq.wq_gemm_w8a16(Xp, q16, fmt, s16, Yp), flush)
+        f = 2.0 * 2048 * N * K
+        out[f"w8a16_{name}_prefill_tflops"] = round(f / (t * 1e-3) / 1e12, 1)
+        out[f"w8a16_{name}_prefill_frac_bf16_peak"] = round(
+            f / (t * 1e-3) / 1e12 / pk["bf16_tflops"], 3)
+    del W16, Xd, Xp, Yd, Yp, q16, s16
+    torch.cuda.empty_cache()
+
     # GPTQ of a [4096, 4096] bf16 weight (the 7B square projection), factor
     # from 8192 synthetic correlated calibration tokens (numpy, not timed)
     K = 4096
@@ -611,7 +635,13 @@ def profile_case(case):
     70B model, 235 MB of codes, larger than L2; three launches), decode-step =
     two warm-up steps then one step of the 7B decode workload (its three
     shapes), prefill = W4A16 GEMM 2048 x 11008 x 4096, w8a8 = W8A8 GEMM 4096^3
-    (three launches each)."""
+    (per-token activation quantization + int8 GEMM), fp8 = the same product in
+    FP8 E4M3, decode-m16 = W4A16 decode product on [11008, 4096] at M = 16
+    (tensor-core kernel), quantize = INT4 g128 quantize + pack of the bf16
+    [11008, 4096] weight, kv = KV-cache INT8 of a bf16 cache [64, 8192, 128]
+    (three launches each); gptq = GPTQ of a bf16 [4096, 4096] weight with a
+    synthetic inverse-Hessian factor (one launch); w8a16 = int8 W8A16 on the
+    [11008, 4096] weight at M = 1 then M = 2048 (three launches each)."""
     import bit_gemm_group_b200 as wq
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -648,6 +678,60 @@ def profile_case(case):
         ws = wq.w4a16_workspace(1, N, K, dev)
         for _ in range(3):
             wq.wq_gemm_w4a16(X, c, s, None, N, 128, True, Y, ws)
+    elif case == "decode-m16":
+        wl = WORKLOADS["7b-decode"]
+        W = wl.weight(1).to(dev)
+        N, K = W.shape
+        c, s, z = wq.quantize_pack(W, 128, 4, True)
+        X = wl.activation(16, K).to(dev)
+        Y = torch.empty((16, N), dtype=torch.bfloat16, device=dev)
+        ws = wq.w4a16_workspace(16, N, K, dev)
+        for _ in range(3):
+            wq.wq_gemm_w4a16(X, c, s, None, N, 128, True, Y, ws)
+    elif case == "quantize":
+        W = WORKLOADS["7b-decode"].weight(1).to(dev)
+        N, K = W.shape
+        c = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+        s = torch.empty((N, K // 128), dtype=torch.float16, device=dev)
+        for _ in range(3):
+            wq.wq_quantize_pack(W, 128, 4, True, c, s, None)
+    elif case == "kv":
+        BH, S, D = 64, 8192, 128
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(6)
+        Kc = torch.randn((BH, S, D), generator=gen, device=dev).to(torch.bfloat16)
+        Vc = torch.randn((BH, S, D), generator=gen, device=dev).to(torch.bfloat16)
+        for _ in range(3):
+            wq.quant_kv(Kc, Vc)
+    elif case == "gptq":
+        K = 4096
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(12)
+        A = torch.randn((K, K), generator=gen, device=dev, dtype=torch.float64) / K ** 0.5
+        H = A.T @ A + 0.01 * torch.eye(K, device=dev, dtype=torch.float64)
+        U = torch.linalg.cholesky(torch.linalg.inv(H)).T.contiguous()  # upper, H^-1 = U^T U
+        del A, H
+        W = WORKLOADS["7b-decode"].weight(0).to(dev)
+        wq.gptq_quantize(W, U, True)
+    elif case == "w8a16":
+        W = WORKLOADS["7b-decode"].weight(1).to(dev)
+        N, K = W.shape
+        q, s, _ = wq.quantize_pack(W, K, 8, True)
+        Xd = WORKLOADS["7b-decode"].activation(1, K).to(dev)
+        Xp = WORKLOADS["prefill"].activation(2048, K).to(dev)
+        for _ in range(3):
+            wq.gemm_w8a16(Xd, q, s)
+        for _ in range(3):
+            wq.gemm_w8a16(Xp, q, s)
+    elif case == "fp8":
+        wl = WORKLOADS["w8a8"]
+        W = wl.weight(0).to(dev)
+        fw, fsw = wq.quantize_fp8_rows(W)
+        X = wl.activation(4096, 4096).to(dev)
+        Y = torch.empty((4096, 4096), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty((wq.wq_w8a8_workspace_bytes(4096, 4096),), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            wq.wq_gemm_fp8(X, fw, fsw, Y, ws)
     elif case == "prefill":
         wl = WORKLOADS["prefill"]
         W = wl.weight(0).to(dev)
@@ -679,7 +763,8 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip the secondary rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
     ap.add_argument("--profile-case",
-                    choices=["decode", "decode-large", "decode-step", "prefill", "w8a8"],
+                    choices=["decode", "decode-large", "decode-step", "decode-m16", "prefill",
+                             "w8a8", "fp8", "quantize", "kv", "gptq", "w8a16"],
                     help="run one kernel 3 times on its workload (for ncu captures) and exit")
     args = ap.parse_args()
     if args.profile_case:

@@ -26,6 +26,11 @@ int launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const double* 
                 void* codes, void* scales, void* zeros, void* ws, cudaStream_t s);
 int launch_gemm_fp8(const void* X, int64_t M, int64_t K, const void* Wq, const void* w_scales,
                     int64_t N, void* Y, void* ws, void* acc_out, cudaStream_t s);
+// W8A16 (int8 or E4M3 per-channel weights, bf16 activations): CUDA-core
+// kernel for M <= kGemvW8a16MaxM, tensor-core GEMM above.
+constexpr int64_t kGemvW8a16MaxM = 4;
+int launch_gemm_w8a16(const void* X, int64_t M, int64_t K, const void* Wq, int w_fmt,
+                      const float* w_scales, int64_t N, void* Y, cudaStream_t s);
 int launch_dequant_int4(const void* codes, const void* scales, const void* zeros, int64_t N,
                         int64_t K, int group_size, int sym, void* out, int out_dtype,
                         cudaStream_t s);

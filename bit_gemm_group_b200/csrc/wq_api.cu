@@ -351,6 +351,24 @@ int wq_gemm_fp8(const void* X, int64_t M, int64_t K, const void* Wq, const void*
   return wq_host::launch_gemm_fp8(X, M, K, Wq, w_scales, N, Y, ws, acc_out, as_stream(stream));
 }
 
+int wq_gemm_w8a16(const void* X, int64_t M, int64_t K, const void* Wq, int w_fmt,
+                  const void* w_scales, int64_t N, void* Y, void* stream) {
+  if (M < 0 || K < 0 || N < 0) return WQ_ERR_ARG;
+  if (w_fmt != WQ_W8_INT8 && w_fmt != WQ_W8_E4M3) return WQ_ERR_ARG;
+  if ((K % 64) != 0) return WQ_ERR_ALIGN;
+  if (M > (int64_t(1) << 31) / 2 || N > (int64_t(1) << 31) / 2 || K > (int64_t(1) << 24))
+    return WQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return WQ_OK;
+  if (K == 0) return WQ_ERR_ARG;
+  if (!X || !Wq || !w_scales || !Y) return WQ_ERR_ARG;
+  if (!aligned16(X) || !aligned16(Wq) || !aligned16(w_scales) || !aligned16(Y))
+    return WQ_ERR_ALIGN;
+  int st = wq_host::ensure_device();
+  if (st != WQ_OK) return st;
+  return wq_host::launch_gemm_w8a16(X, M, K, Wq, w_fmt, static_cast<const float*>(w_scales), N,
+                                    Y, as_stream(stream));
+}
+
 // -------------------------------------------------------------------- GPTQ
 
 size_t wq_gptq_workspace_bytes(int64_t N, int64_t K) {

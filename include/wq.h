@@ -122,6 +122,16 @@ WQ_API int wq_dequant(const void *codes, const void *scales, const void *zeros,
  * larger M runs the tensor-core GEMM.
  * Requires K % 128 == 0 and N % 8 == 0.
  *
+ * Stream order: the CUDA-core decode kernel is launched as a programmatic
+ * dependent of the kernel before it on the stream.  It starts streaming
+ * codes and scales (and zeros) while that kernel is still finishing, and
+ * reads X, and writes Y, only after it has completed.  Weights are inputs
+ * that do not change from call to call: they must not be written by the
+ * kernel immediately preceding the call on the same stream while that kernel
+ * itself triggers its dependents early (of this library's kernels only this
+ * decode kernel does, and it writes no weights; a kernel that does not
+ * trigger lets the call start only once all its blocks have exited).
+ *
  * ws / ws_bytes: device workspace of wq_w4a16_workspace_bytes(M, N, K) bytes
  * (0 for M > 16, where ws may be NULL).  Fill it with zeros once before its
  * first use (e.g. cudaMemset); every call that completes leaves the part that
@@ -275,6 +285,24 @@ WQ_API int wq_quant_kv(const void *K, const void *V, int dtype, int64_t BH, int6
  */
 WQ_API int wq_quantize_fp8_rows(const void *A, int a_dtype, int64_t R, int64_t K,
                                 void *q, void *scales, void *stream);
+
+/*
+ * wq_gemm_w8a16 -- W8A16 ([P4] sec. 2.3 naming table: 8-bit weights with
+ * 16-bit activations; the weight is expanded to the activation type inside
+ * the product, never written back): Y = bf16(w_scales[n] * acc[m, n]) with
+ * acc = sum_k X[m, k] * value(Wq[n, k]) accumulated in fp32.
+ * X bf16 [M, K]; Wq [N, K] per-output-channel codes, w_fmt WQ_W8_INT8 (int8
+ * codes with fp32 scales, as wq_quantize_pack with bits 8 writes them) or
+ * WQ_W8_E4M3 (E4M3 codes with fp32 scales, as wq_quantize_fp8_rows writes
+ * them); w_scales fp32 [N]; Y bf16 [M, N].  Every code value is exact in
+ * bf16, so the expanded weight is not rounded.  M <= 4 runs on the CUDA
+ * cores (every weight byte streamed once), larger M on the tensor cores
+ * (tcgen05.mma kind::f16).  Requires K % 64 == 0; all pointers 16-byte
+ * aligned.
+ */
+enum { WQ_W8_INT8 = 0, WQ_W8_E4M3 = 1 };
+WQ_API int wq_gemm_w8a16(const void *X, int64_t M, int64_t K, const void *Wq, int w_fmt,
+                         const void *w_scales, int64_t N, void *Y, void *stream);
 
 /*
  * wq_gemm_fp8 -- Y = bf16(acc * sx[m] * w_scales[n]) with acc[m, n] =
