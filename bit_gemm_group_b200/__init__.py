@@ -152,6 +152,19 @@ def _bf16(t, what):
     return _ptr(t)
 
 
+def _fits(t, nbytes, what):
+    """Refuse a buffer smaller than the bytes the call will touch: the C ABI
+    receives bare pointers and cannot check their extent."""
+    if isinstance(t, torch.Tensor):
+        have = t.numel() * t.element_size()
+        if have < nbytes:
+            raise WQError(WQ_ERR_ARG, f"{what} holds {have} bytes, the call needs {int(nbytes)}")
+
+
+def _groups(K, group_size):
+    return K // group_size if group_size > 0 and K % group_size == 0 else 0
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -165,6 +178,14 @@ _DTYPE_TAG = {torch.float32: WQ_F32, torch.bfloat16: WQ_BF16, torch.float16: WQ_
 
 def wq_quantize_pack(W, group_size, bits, sym, codes, scales, zeros=None, stream=None):
     N, K = W.shape
+    if bits == 4:
+        G = _groups(K, group_size)
+        _fits(codes, N * K // 2, "codes")
+        _fits(scales, 2 * N * G, "scales")
+        _fits(zeros, 2 * N * G, "zeros")
+    elif bits == 8:
+        _fits(codes, N * K, "codes")
+        _fits(scales, 4 * N, "scales")
     st = lib().wq_quantize_pack(_ptr(W), _DTYPE_TAG.get(W.dtype, -1), N, K, group_size, bits,
                                 int(bool(sym)), _ptr(codes), _ptr(scales), _ptr(zeros),
                                 _stream(stream))
@@ -173,6 +194,15 @@ def wq_quantize_pack(W, group_size, bits, sym, codes, scales, zeros=None, stream
 
 def wq_dequant(codes, scales, zeros, N, K, group_size, bits, sym, out, stream=None):
     tag = _DTYPE_TAG.get(out.dtype, -1)
+    if bits == 4:
+        G = _groups(K, group_size)
+        _fits(codes, N * K // 2, "codes")
+        _fits(scales, 2 * N * G, "scales")
+        _fits(zeros, 2 * N * G, "zeros")
+    elif bits == 8:
+        _fits(codes, N * K, "codes")
+        _fits(scales, 4 * N, "scales")
+    _fits(out, N * K * out.element_size(), "out")
     st = lib().wq_dequant(_ptr(codes), _ptr(scales), _ptr(zeros), N, K, group_size, bits,
                           int(bool(sym)), _ptr(out), tag, _stream(stream))
     _check(st, "wq_dequant")
@@ -184,6 +214,11 @@ def wq_w4a16_workspace_bytes(M, N, K):
 
 def wq_gemm_w4a16(X, codes, scales, zeros, N, group_size, sym, Y, ws=None, stream=None):
     M, K = X.shape
+    G = _groups(K, group_size)
+    _fits(codes, N * K // 2, "codes")
+    _fits(scales, 2 * N * G, "scales")
+    _fits(zeros, 2 * N * G, "zeros")
+    _fits(Y, 2 * M * N, "Y")
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     st = lib().wq_gemm_w4a16(_bf16(X, "X"), M, K, _ptr(codes), _ptr(scales), _ptr(zeros), N,
                              group_size, int(bool(sym)), _bf16(Y, "Y"), _ptr(ws), ws_bytes,
@@ -196,6 +231,11 @@ def wq_gemm_w4a16_noalloc(X, codes, scales, zeros, N, group_size, sym, Y, stream
     allocation.  Overlapping calls race; the first call per device must not
     be inside a stream capture."""
     M, K = X.shape
+    G = _groups(K, group_size)
+    _fits(codes, N * K // 2, "codes")
+    _fits(scales, 2 * N * G, "scales")
+    _fits(zeros, 2 * N * G, "zeros")
+    _fits(Y, 2 * M * N, "Y")
     st = lib().wq_gemm_w4a16_noalloc(_bf16(X, "X"), M, K, _ptr(codes), _ptr(scales),
                                      _ptr(zeros), N, group_size, int(bool(sym)), _bf16(Y, "Y"),
                                      _stream(stream))
@@ -204,6 +244,8 @@ def wq_gemm_w4a16_noalloc(X, codes, scales, zeros, N, group_size, sym, Y, stream
 
 def wq_quant_act_i8(X, q, s, stream=None):
     M, K = X.shape
+    _fits(q, M * K, "q")
+    _fits(s, 4 * M, "s")
     st = lib().wq_quant_act_i8(_bf16(X, "X"), M, K, _ptr(q), _ptr(s), _stream(stream))
     _check(st, "wq_quant_act_i8")
 
@@ -215,6 +257,10 @@ def wq_w8a8_workspace_bytes(M, K):
 def wq_gemm_w8a8(X, Wq, w_scales, Y, ws, acc_out=None, stream=None):
     M, K = X.shape
     N = Wq.shape[0]
+    _fits(Wq, N * K, "Wq")
+    _fits(w_scales, 4 * N, "w_scales")
+    _fits(Y, 2 * M * N, "Y")
+    _fits(acc_out, 4 * M * N, "acc_out")
     st = lib().wq_gemm_w8a8(_bf16(X, "X"), M, K, _ptr(Wq), _ptr(w_scales), N, _bf16(Y, "Y"),
                             _ptr(ws), ws.numel() * ws.element_size(), _ptr(acc_out),
                             _stream(stream))
@@ -223,12 +269,16 @@ def wq_gemm_w8a8(X, Wq, w_scales, Y, ws, acc_out=None, stream=None):
 
 def wq_channel_absmax(A, out, stream=None):
     R, K = A.shape
+    _fits(out, 4 * K, "out")
     st = lib().wq_channel_absmax(_ptr(A), _DTYPE_TAG.get(A.dtype, -1), R, K, _ptr(out),
                                  _stream(stream))
     _check(st, "wq_channel_absmax")
 
 
 def wq_smooth_scales(act_absmax, w_absmax, alpha, s, stream=None):
+    K = act_absmax.numel()
+    _fits(w_absmax, 4 * K, "w_absmax")
+    _fits(s, 4 * K, "s")
     st = lib().wq_smooth_scales(_ptr(act_absmax), _ptr(w_absmax), act_absmax.numel(),
                                 float(alpha), _ptr(s), _stream(stream))
     _check(st, "wq_smooth_scales")
@@ -236,6 +286,9 @@ def wq_smooth_scales(act_absmax, w_absmax, alpha, s, stream=None):
 
 def wq_quantize_i8_smooth(W, s, q, scales, stream=None):
     N, K = W.shape
+    _fits(s, 4 * K, "s")
+    _fits(q, N * K, "q")
+    _fits(scales, 4 * N, "scales")
     st = lib().wq_quantize_i8_smooth(_ptr(W), _DTYPE_TAG.get(W.dtype, -1), N, K, _ptr(s),
                                      _ptr(q), _ptr(scales), _stream(stream))
     _check(st, "wq_quantize_i8_smooth")
@@ -243,6 +296,9 @@ def wq_quantize_i8_smooth(W, s, q, scales, stream=None):
 
 def wq_quant_act_i8_smooth(X, s, q, sx, stream=None):
     M, K = X.shape
+    _fits(s, 4 * K, "s")
+    _fits(q, M * K, "q")
+    _fits(sx, 4 * M, "sx")
     st = lib().wq_quant_act_i8_smooth(_bf16(X, "X"), M, K, _ptr(s), _ptr(q), _ptr(sx),
                                       _stream(stream))
     _check(st, "wq_quant_act_i8_smooth")
@@ -251,6 +307,11 @@ def wq_quant_act_i8_smooth(X, s, q, sx, stream=None):
 def wq_gemm_w8a8_smooth(X, Wq, w_scales, s, Y, ws, acc_out=None, stream=None):
     M, K = X.shape
     N = Wq.shape[0]
+    _fits(s, 4 * K, "s")
+    _fits(Wq, N * K, "Wq")
+    _fits(w_scales, 4 * N, "w_scales")
+    _fits(Y, 2 * M * N, "Y")
+    _fits(acc_out, 4 * M * N, "acc_out")
     st = lib().wq_gemm_w8a8_smooth(_bf16(X, "X"), M, K, _ptr(Wq), _ptr(w_scales), _ptr(s), N,
                                    _bf16(Y, "Y"), _ptr(ws), ws.numel() * ws.element_size(),
                                    _ptr(acc_out), _stream(stream))
@@ -259,6 +320,11 @@ def wq_gemm_w8a8_smooth(X, Wq, w_scales, s, Y, ws, acc_out=None, stream=None):
 
 def wq_quant_kv(K, V, qk, sk, qv, sv, stream=None):
     BH, S, D = K.shape
+    _fits(V, K.numel() * K.element_size(), "V")
+    _fits(qk, BH * S * D, "qk")
+    _fits(qv, BH * S * D, "qv")
+    _fits(sk, 4 * BH * D, "sk")
+    _fits(sv, 4 * BH * S, "sv")
     st = lib().wq_quant_kv(_ptr(K), _ptr(V), _DTYPE_TAG.get(K.dtype, -1), BH, S, D, _ptr(qk),
                            _ptr(sk), _ptr(qv), _ptr(sv), _stream(stream))
     _check(st, "wq_quant_kv")
@@ -266,6 +332,8 @@ def wq_quant_kv(K, V, qk, sk, qv, sv, stream=None):
 
 def wq_quantize_fp8_rows(A, q, scales, stream=None):
     R, K = A.shape
+    _fits(q, R * K, "q")
+    _fits(scales, 4 * R, "scales")
     st = lib().wq_quantize_fp8_rows(_ptr(A), _DTYPE_TAG.get(A.dtype, -1), R, K, _ptr(q),
                                     _ptr(scales), _stream(stream))
     _check(st, "wq_quantize_fp8_rows")
@@ -274,6 +342,10 @@ def wq_quantize_fp8_rows(A, q, scales, stream=None):
 def wq_gemm_fp8(X, Wq, w_scales, Y, ws, acc_out=None, stream=None):
     M, K = X.shape
     N = Wq.shape[0]
+    _fits(Wq, N * K, "Wq")
+    _fits(w_scales, 4 * N, "w_scales")
+    _fits(Y, 2 * M * N, "Y")
+    _fits(acc_out, 4 * M * N, "acc_out")
     st = lib().wq_gemm_fp8(_bf16(X, "X"), M, K, _ptr(Wq), _ptr(w_scales), N, _bf16(Y, "Y"),
                            _ptr(ws), ws.numel() * ws.element_size(), _ptr(acc_out),
                            _stream(stream))
@@ -286,6 +358,9 @@ WQ_W8_INT8, WQ_W8_E4M3 = 0, 1
 def wq_gemm_w8a16(X, Wq, w_fmt, w_scales, Y, stream=None):
     M, K = X.shape
     N = Wq.shape[0]
+    _fits(Wq, N * K, "Wq")
+    _fits(w_scales, 4 * N, "w_scales")
+    _fits(Y, 2 * M * N, "Y")
     st = lib().wq_gemm_w8a16(_bf16(X, "X"), M, K, _ptr(Wq), int(w_fmt), _ptr(w_scales), N,
                              _bf16(Y, "Y"), _stream(stream))
     _check(st, "wq_gemm_w8a16")
@@ -293,6 +368,11 @@ def wq_gemm_w8a16(X, Wq, w_fmt, w_scales, Y, stream=None):
 
 def wq_gptq_quantize(W, U, group_size, sym, codes, scales, zeros, ws, stream=None):
     N, K = W.shape
+    G = _groups(K, group_size)
+    _fits(U, 8 * K * K, "U")
+    _fits(codes, N * K // 2, "codes")
+    _fits(scales, 2 * N * G, "scales")
+    _fits(zeros, 2 * N * G, "zeros")
     st = lib().wq_gptq_quantize(_ptr(W), _DTYPE_TAG.get(W.dtype, -1), N, K, _ptr(U), group_size,
                                 int(bool(sym)), _ptr(codes), _ptr(scales), _ptr(zeros),
                                 _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))

@@ -168,3 +168,60 @@ def test_binding_rejects_non_bf16_activations():
     assert e.value.status == wq.WQ_ERR_ARG and "bfloat16" in str(e.value)
     with pytest.raises(wq.WQError):
         wq.wq_gemm_w4a16(X16, q, s, None, 8, 128, True, X16)
+
+
+def test_binding_refuses_short_buffers():
+    """Every buffer's extent is checked against the sizes the call passes,
+    before any pointer reaches the library (the C ABI cannot see extents)."""
+    X = torch.zeros((4, 256), dtype=torch.bfloat16)
+    codes = torch.zeros((8, 64), dtype=torch.uint8)        # needs [8, 128]
+    scales = torch.zeros((8, 2), dtype=torch.float16)
+    Y = torch.zeros((4, 8), dtype=torch.bfloat16)
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_gemm_w4a16(X, codes, scales, None, 8, 128, True, Y)
+    assert e.value.status == wq.WQ_ERR_ARG and "codes" in str(e.value)
+    W = torch.zeros((8, 256), dtype=torch.bfloat16)
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_quantize_pack(W, 128, 4, True, torch.zeros((8, 128), dtype=torch.uint8),
+                            torch.zeros((8, 1), dtype=torch.float16))
+    assert "scales" in str(e.value)
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_gemm_w8a16(X, torch.zeros((8, 256), dtype=torch.int8), 0,
+                         torch.zeros(8, dtype=torch.float32), torch.zeros((4, 4), dtype=torch.bfloat16))
+    assert "Y" in str(e.value)
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_quant_act_i8(X, torch.zeros((4, 256), dtype=torch.int8), torch.zeros(3))
+    assert "s holds" in str(e.value)
+
+
+def test_helpers_allocate_what_the_calls_touch():
+    """The allocating helpers pass the extent checks: with CPU tensors every
+    call stops only at the device check (no CPU fallback)."""
+    N, K, M = 16, 256, 4
+    bf = torch.bfloat16
+    W, X = torch.zeros(N, K, dtype=bf), torch.zeros(M, K, dtype=bf)
+    codes = torch.zeros(N, K // 2, dtype=torch.uint8)
+    sc = torch.zeros(N, K // 128, dtype=torch.float16)
+    q8, s8 = torch.zeros(N, K, dtype=torch.int8), torch.zeros(N)
+    U = torch.zeros(K, K, dtype=torch.float64)
+    calls = [
+        lambda: wq.quantize_pack(W, 128, 4, True), lambda: wq.quantize_pack(W, 128, 4, False),
+        lambda: wq.quantize_pack(W, K, 8, True),
+        lambda: wq.dequant(codes, sc, sc, K, 128, 4, False, torch.float32),
+        lambda: wq.dequant(q8, s8, None, K, K, 8, True, bf),
+        lambda: wq.gemm_w4a16(X, codes, sc, sc, 128, False),
+        lambda: wq.quant_act_i8(X), lambda: wq.gemm_w8a8(X, q8, s8, want_acc=True),
+        lambda: wq.channel_absmax(X), lambda: wq.smooth_scales(torch.zeros(K), torch.zeros(K)),
+        lambda: wq.quantize_i8_smooth(W, torch.zeros(K)),
+        lambda: wq.quant_act_i8_smooth(X, torch.zeros(K)),
+        lambda: wq.gemm_w8a8_smooth(X, q8, s8, torch.zeros(K)),
+        lambda: wq.quant_kv(torch.zeros(2, 8, 128, dtype=bf), torch.zeros(2, 8, 128, dtype=bf)),
+        lambda: wq.quantize_fp8_rows(W),
+        lambda: wq.gemm_fp8(X, torch.zeros(N, K, dtype=torch.uint8), s8),
+        lambda: wq.gemm_w8a16(X, q8, s8),
+        lambda: wq.gptq_quantize(W, U, True), lambda: wq.gptq_quantize(W, U, False),
+    ]
+    for call in calls:
+        with pytest.raises(wq.WQError) as e:
+            call()
+        assert "CUDA device" in str(e.value)
