@@ -37,7 +37,7 @@ def _worker(rank, world, port, out):
 
 def test_two_ranks_agree_on_the_slowest_time():
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_worker, args=(2, port, out), nprocs=2, join=True,
                            start_method="spawn")
