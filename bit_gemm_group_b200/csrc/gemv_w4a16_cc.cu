@@ -14,9 +14,9 @@
 //
 // Exact integer inner products.  Each CTA first rewrites X per (row m, group
 // g) as integers x' = rint(x * 2^e), e chosen so that the group's largest |x|
-// lands in [2^12, 2^13) (bf16 values that large are integers there already;
-// only elements below 2^-8 of the group maximum lose bits, at most 2^-13 of
-// the maximum each).  x' = 128 h + l with h in [-64, 64] and l in [0, 127]
+// lands in [2^12, 2^13) (bf16 values down to 2^-5 of the group maximum are
+// integers there already; smaller ones lose bits, at most 2^-13 of the
+// maximum each).  x' = 128 h + l with h in [-64, 64] and l in [0, 127]
 // gives two int8 limbs.  A 32-bit code word holds elements e0..e7 (low nibble
 // of byte b = e_2b): w & 0x0F0F0F0F holds the even elements as bytes and
 // (w >> 4) & 0x0F0F0F0F the odd ones, so four DP4A instructions take the word

@@ -1,0 +1,89 @@
+"""Host restatement of the CUDA-core decode kernel's arithmetic (W4A16,
+M <= 4): each (activation row, 128-group) of X becomes integers
+x' = rint(x 2^e) with the group's max |x'| in [2^12, 2^13), split into int8
+limbs x' = 128 h + l; the group's dot product with the codes is an exact
+integer, scaled once by s 2^-e.  These tests pin the limb ranges DP4A needs,
+the exactness of the integer sums and the error bound against the fp64
+product."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import bf16_bits, make_activation, make_weight
+
+
+def prepare(x):
+    """x: float32 [G, 128] (bf16 values) -> (x' int64, e int)."""
+    amax = np.abs(x).max(axis=1).astype(np.float32)
+    E = (amax.view(np.uint32) >> 23).astype(np.int64)
+    e = np.clip(139 - E, -126, 126)
+    xi = np.rint(x.astype(np.float64) * np.exp2(e)[:, None]).astype(np.int64)
+    return xi, e
+
+
+def test_limbs_fit_dp4a():
+    rng = np.random.default_rng(0)
+    for scale in (1e-6, 1e-2, 1.0, 50.0, 3e4):
+        x = oracle.bf16_to_f32(oracle.f32_to_bf16(
+            (rng.standard_normal((400, 128)) * scale).astype(np.float32))).reshape(400, 128)
+        xi, e = prepare(x)
+        m = np.abs(xi).max(axis=1)
+        assert ((m >= 2 ** 12) & (m <= 2 ** 13)).all()   # the rounded max may reach 2^13
+        h, l = xi >> 7, xi & 127
+        assert np.array_equal(128 * h + l, xi)
+        assert h.min() >= -64 and h.max() <= 64 and l.min() >= 0 and l.max() <= 127
+
+
+def test_integer_sums_are_exact_and_small():
+    rng = np.random.default_rng(1)
+    x = oracle.bf16_to_f32(oracle.f32_to_bf16(rng.standard_normal((200, 128)).astype(np.float32))).reshape(200, 128)
+    xi, _ = prepare(x)
+    u = rng.integers(0, 16, (200, 128))
+    z = rng.integers(0, 16, (200, 1))
+    h, l = xi >> 7, xi & 127
+    per_lane = 128 * (u[:, :32] * h[:, :32]).sum(1) + (u[:, :32] * l[:, :32]).sum(1)
+    assert np.abs(per_lane).max() < 2 ** 22     # one lane's 32 elements: exact in int32 and fp32
+    t = 128 * (u * h).sum(1) + (u * l).sum(1) - z[:, 0] * xi.sum(1)
+    assert np.array_equal(t, ((u - z) * xi).sum(1))
+
+
+@pytest.mark.parametrize("sym", [True, False])
+def test_product_error_within_the_stated_bound(sym):
+    """Only elements below 2^-5 of their group maximum lose bits, each by at
+    most 2^-13 of the maximum (a group holding an outlier dimension rounds
+    nearly all its other elements); the product stays inside the 2e-3
+    row-normalised tolerance against the fp64 oracle with a wide margin."""
+    N, K, M = 64, 1024, 2
+    W = make_weight(N, K, 0.02, seed=4, outlier_frac=0.01, outlier_scale=30.0, dtype=torch.float32)
+    codes, scales, zeros, st = oracle.quantize_int4(W.numpy(), 128, sym)
+    assert st == oracle.OK
+    X = make_activation(M, K, seed=5, outlier_dims=6)
+    Xb = bf16_bits(X)
+    ref, _ = oracle.gemm_w4a16(Xb, codes, scales, zeros, 128, sym)
+    x = oracle.bf16_to_f32(Xb).reshape(M, K)
+    u = np.zeros((N, K), np.int64)
+    u[:, 0::2] = codes & 15
+    u[:, 1::2] = codes >> 4
+    s = oracle.f16_to_f32(scales).reshape(N, K // 128).astype(np.float32)
+    zf = np.full((N, K // 128), 8) if sym else oracle.f16_to_f32(zeros).reshape(N, K // 128)
+    Y = np.zeros((M, N))
+    for m in range(M):
+        xi, e = prepare(x[m].reshape(K // 128, 128))
+        for g in range(K // 128):
+            ug = u[:, g * 128:(g + 1) * 128] - zf[:, g:g + 1].astype(np.int64)
+            t = (ug * xi[g]).sum(1)                       # exact integers
+            Y[m] += (t.astype(np.float32) * (s[:, g] * np.float32(2.0 ** -e[g]))).astype(np.float64)
+    err = np.abs(Y - ref).max(axis=1) / np.linalg.norm(ref, axis=1)
+    assert err.max() < 1e-3
+
+
+def test_exact_down_to_two_to_the_minus_five_of_the_maximum():
+    rng = np.random.default_rng(2)
+    x = oracle.bf16_to_f32(oracle.f32_to_bf16(rng.standard_normal((2000, 128)).astype(np.float32))).reshape(2000, 128)
+    xi, e = prepare(x)
+    amax = np.abs(x).max(axis=1, keepdims=True)
+    err = np.abs(x - xi * np.exp2(-e)[:, None])
+    assert (err[np.abs(x) >= amax * 2.0 ** -5] == 0).all()
+    assert (err <= amax * 2.0 ** -13).all()
+    assert (err > 0).any()
