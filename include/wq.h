@@ -12,7 +12,8 @@
  *
  * Conventions for every entry point:
  *   - All tensor arguments are DEVICE pointers to row-major buffers that the
- *     caller allocates and owns.  The library keeps no pointer after return.
+ *     caller allocates and owns, on the current CUDA device (the one the
+ *     stream belongs to).  The library keeps no pointer after return.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Work is enqueued asynchronously on that stream.
  *   - The return value reports host-side argument validation and launch
