@@ -522,13 +522,7 @@ size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 }
 
 bool decode_on_cuda_cores(int64_t M, int64_t N, int64_t K) {
-  if (M > kGemvCcMaxM || gemv_cc_depth(M, K) == 0) return false;
-  if (M <= 2) return true;
-  // Three or four activation rows cost the CUDA-core kernel about twice the
-  // issue slots of one row: it still wins on small matrices, where the
-  // tensor-core kernel's fixed latency dominates (4096 x 4096: 12 vs 15 us),
-  // and loses on large ones (28672 x 8192: 67 vs 56 us).
-  return K <= 8192 && N * K <= (int64_t(1) << 26);
+  return M <= kGemvCcMaxM && gemv_cc_fits(M, N, K);
 }
 
 int launch_decode_w4a16(const void* X, int64_t M, int64_t K, const void* codes,

@@ -8,402 +8,438 @@
 // bandwidth; sec. 2.3 W4A16; "大模型量化技术定义与主流方案解析" sec. 四: the
 // weight is expanded inside the product and never written back.)
 //
-// At M <= 4 the arithmetic per weight byte is small enough for the CUDA cores,
-// and a streaming kernel keeps every SM's loads in flight from its first cycle
-// to its last, with none of the tensor-core path's hand-offs between warps.
+// At M <= 4 there is too little arithmetic per weight byte for the tensor
+// cores to help: the kernel is a stream, and what bounds it is how many issue
+// slots it spends per byte and how many bytes it keeps in flight.
 //
-// Exact integer inner products.  Each CTA first rewrites X per (row m, group
-// g) as integers x' = rint(x * 2^e), e chosen so that the group's largest |x|
-// lands in [2^12, 2^13) (bf16 values down to 2^-5 of the group maximum are
-// integers there already; smaller ones lose bits, at most 2^-13 of the
-// maximum each).  x' = 128 h + l with h in [-64, 64] and l in [0, 127]
-// gives two int8 limbs.  A 32-bit code word holds elements e0..e7 (low nibble
-// of byte b = e_2b): w & 0x0F0F0F0F holds the even elements as bytes and
-// (w >> 4) & 0x0F0F0F0F the odd ones, so four DP4A instructions take the word
-// against the limbs of X.  Per lane (32 elements of one group) the sum
-//   sum (u - z) x' = 128 sum u h + sum u l - z sum x'
-// is exact in int32 (below 2^22), and only s * 2^-e * (that) is rounded, in
-// fp32, when it is accumulated.
+// Exact integer inner products.  X is rewritten per (activation row m,
+// group g of 128 along K) as integers x' = rint(x * 2^e), e chosen so that
+// the group's largest |x| lands in [2^12, 2^13): bf16 values down to 2^-5 of
+// the group maximum are integers there already, smaller ones lose bits (at
+// most 2^-13 of the maximum each).  x' fits in 16 bits, and a pair of them
+// is one operand of DP2A.  A 32-bit code word holds elements e0..e7 (the low
+// nibble of byte b is e_2b): w & 0x0F0F0F0F holds the even elements as bytes
+// and w & 0xF0F0F0F0 sixteen times the odd ones, so four DP2A take the word
+// against X (the odd sum is exactly divisible by 16).  A group's
+//   sum (u - z) x' = sum u x' - z sum x'
+// is exact in int32 (below 2^24, so also exact as a float) and only
+// s * 2^-e * (that) is rounded, in fp32.
 //
-// Work split.  An item is (block of R = 4 weight rows, 1024-wide K chunk);
-// lane l of a warp takes elements [32 l, 32 l + 32) of the chunk, i.e. 16
-// coalesced bytes of codes per row.  CTA c of the P-CTA grid (one per SM)
-// owns row blocks [c NB / P, (c + 1) NB / P), so SMs differ by at most one row
-// block; its I_c items, numbered row-block-major, are split into 16 equal
-// contiguous ranges, one per warp.  A row block that one warp covers entirely
-// is written straight to Y; the partial sums of the (at most 16) row blocks
-// that straddle two warps' ranges go to shared memory and are added in warp
-// order after the CTA's barrier (deterministic, no global atomics).
+// Work split.  An item is (8 weight rows, one 1024-wide K chunk): 512
+// contiguous bytes of codes per row, 16 per lane, lane l covering elements
+// [32 l, 32 l + 32) of the chunk (a quarter of group l / 4).  CTA c of the
+// one-per-SM grid owns the 4-row blocks [c NB / P, (c + 1) NB / P), so SMs
+// differ by at most four rows.  Its items are numbered chunk-major (all of the
+// CTA's row tiles for chunk 0, then chunk 1, ...) and split into equal
+// contiguous ranges, one per warp, so a warp keeps one chunk's X in registers
+// for many items and converts X only when its chunk changes.  Each item ends
+// in a transposed reduction: the 4 lanes of a group exchange row sums in two
+// shuffle rounds (each lane keeps 2 of the 8 rows, as exact integers), apply
+// the group's scale and zero point to those, and three more rounds sum the 8
+// groups of the chunk.  The chunk's partial sum of each row lands in shared
+// memory; after one barrier the CTA adds a row's chunk partials in chunk
+// order (deterministic, no atomics, no workspace).
 //
-// Data movement.  Codes land through a per-warp ring of D items in shared
-// memory (cp.async, 16 bytes per lane and row); each lane reads back exactly
-// the bytes it copied, so the only synchronisation is the lane's own
-// cp.async group count, and D - 1 items per warp are in flight while one is
-// computed.  The CTA prepares X for all K while the first items stream in and
-// keeps it in shared memory in lane order, so every read of it is a
-// conflict-free 16-byte load.
+// Data movement.  Each warp has its own ring of D item slots in shared
+// memory, filled by TMA (one 2D box of 4 rows x 512 bytes per 4 rows, issued
+// by one lane) that completes on the slot's mbarrier.  A warp refills a slot
+// as soon as it has read its codes into registers, before computing them, so
+// D items per warp are in flight almost all the time.  The launch shape
+// (warps per CTA, ring depth) depends on the matrix size (cc_config).
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace wq {
 namespace gemv_cc {
 
-constexpr int THREADS = 512;
-constexpr int WARPS = THREADS / 32;
 constexpr int CHUNK = 1024;               // K elements per item: 32 per lane
-constexpr int R = 4;                      // weight rows per item
-constexpr int ITEM_BYTES = R * CHUNK / 2; // codes of one item (2 KB)
-constexpr int MAXD = 6;
+constexpr int RB = 8;                     // weight rows per item
+constexpr int ROW_BYTES = CHUNK / 2;      // codes of one row of an item
+constexpr int ITEM_BYTES = RB * ROW_BYTES;
+constexpr int BOX_BYTES = 4 * ROW_BYTES;  // one TMA box: 4 rows of an item
 constexpr int SMEM_LIMIT = 227 * 1024;
-constexpr int MT_MAX = 4;
+constexpr uint32_t MAGIC = 0x4B400000u;   // bit pattern of 1.5 * 2^23
 
-// sum of the four byte products a_i * b_i plus c; a unsigned, b signed bytes
-__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+// d = c + a.h0 * b.b0 + a.h1 * b.b1 (lo: bytes 0, 1 of b; hi: bytes 2, 3);
+// a holds two signed 16-bit values, b four unsigned bytes
+__device__ __forceinline__ int dp2a_lo(uint32_t a, uint32_t b, int c) {
   int d;
-  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
-__device__ __forceinline__ uint32_t pack_bytes(int b0, int b1, int b2, int b3) {
-  return (uint32_t(b0) & 0xFFu) | ((uint32_t(b1) & 0xFFu) << 8) | ((uint32_t(b2) & 0xFFu) << 16) |
-         (uint32_t(b3) << 24);
+__device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src) {
-  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
-  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(d), "l"(src)
-               : "memory");
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
 }
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
+// elementwise max(|a|, |b|) of two bf16 pairs (the result's sign bits are
+// not meaningful)
+__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(tc::smem_u32(p)));
+  return v;
 }
-
-// ------------------------------------------------------------------ X prep
-// The CTA's threads rewrite X [M, K] bf16 into shared memory, one 8-element
-// block (row m, elements 8 kb .. 8 kb + 7) per thread and round; the 16 blocks
-// of a group sit in one half-warp and the 4 blocks of a lane's 32 elements in
-// one quad.  Block (q, l) of chunk c -- elements c * CHUNK + 32 l + 8 q .. --
-// becomes 16 bytes {even h, even l, odd h, odd l} (limb bytes of elements
-// 0, 2, 4, 6 and 1, 3, 5, 7) at xs[(m C + c) 128 + 32 q + l]; sx[(m C + c) 32
-// + l] = the lane's sum of x'; inv[m G + g] = 2^-e.
-__device__ __forceinline__ void prepare_x(const __nv_bfloat16* __restrict__ X, int M, int K,
-                                          int C, uint4* __restrict__ xs, int* __restrict__ sx,
-                                          float* __restrict__ invs) {
-  const int kb8 = K / 8;
-  const int total = M * kb8;
-  for (int base = 0; base < total; base += blockDim.x) {
-    const int i = base + threadIdx.x;
-    const bool act = i < total;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (act) v = __ldg(reinterpret_cast<const uint4*>(X) + i);
-    float x[8];
-    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      x[2 * r] = __uint_as_float(wv[r] << 16);
-      x[2 * r + 1] = __uint_as_float(wv[r] & 0xFFFF0000u);
-    }
-    float amax = 0.f;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) amax = fmaxf(amax, fabsf(x[r]));
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    // amax in [2^(E-127), 2^(E-126)) for its biased exponent E; 2^e puts it
-    // in [2^12, 2^13).  A zero (or subnormal) group takes the largest step.
-    const int E = int(__float_as_uint(amax) >> 23);
-    const int e = max(min(139 - E, 126), -126);
-    const float sc = __uint_as_float(uint32_t(127 + e) << 23);
-    int xi[8], hi[8], lo[8], sum = 0;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      xi[r] = __float2int_rn(x[r] * sc);  // |xi| <= 2^13
-      hi[r] = xi[r] >> 7;                 // floor: xi = 128 hi + lo, lo in [0, 127]
-      lo[r] = xi[r] & 127;
-      sum += xi[r];
-    }
-    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-    if (act) {
-      const int m = i / kb8, kb = i - m * kb8;
-      const int c = kb >> 7, l = (kb >> 2) & 31, q = kb & 3;
-      uint4 o;
-      o.x = pack_bytes(hi[0], hi[2], hi[4], hi[6]);
-      o.y = pack_bytes(lo[0], lo[2], lo[4], lo[6]);
-      o.z = pack_bytes(hi[1], hi[3], hi[5], hi[7]);
-      o.w = pack_bytes(lo[1], lo[3], lo[5], lo[7]);
-      xs[(m * C + c) * 128 + q * 32 + l] = o;
-      if (q == 0) sx[(m * C + c) * 32 + l] = sum;
-      if ((threadIdx.x & 15) == 0) invs[i >> 4] = __uint_as_float(uint32_t(127 - e) << 23);
-    }
-  }
-}
-
-// ------------------------------------------------------------------ product
 struct Shape {
-  int M, N, K, G, C, NB;  // NB = row blocks, C = chunks per row
+  int M, N, K, G, C;  // G = groups per row, C = chunks per row
+  int NB;             // 4-row blocks
+  int rows_max;       // rows of the largest CTA range (partials stride)
   int sym;
 };
 
-// Position of an item: row block b, chunk c.
-struct Pos {
-  int b, c;
-  __device__ __forceinline__ void next(int C) {
-    if (++c == C) {
-      c = 0;
-      ++b;
+// An item: chunk c, row tile t of the CTA (chunk-major order).
+struct Item {
+  int c, t;
+  __device__ __forceinline__ void next(int T) {
+    if (++t == T) {
+      t = 0;
+      ++c;
     }
   }
 };
 
-// Copies the codes of the item at p (when `live`) into ring slot `slot` and
-// closes one cp.async group (an empty one otherwise).  Items whose R rows all
-// exist take the path without per-row checks.
-__device__ __forceinline__ void issue_item(uint4* __restrict__ ring_w, int slot,
-                                           const uint8_t* __restrict__ codes, Pos p, bool live,
-                                           const Shape& sh, int lane) {
-  const int k = p.c * CHUNK + lane * 32;
-  if (live && k < sh.K) {
-    const size_t rowb = size_t(sh.K >> 1);
-    const uint8_t* src = codes + size_t(p.b * R) * rowb + (k >> 1);
-    uint4* dst = ring_w + slot * (R * 32) + lane;
-    if (p.b * R + R <= sh.N) {
+// Per-lane view of one chunk of X (activation rows m < MT): for each of the
+// lane's 4 code words q, x' of its even elements {0, 2}, {4, 6} and odd
+// elements {1, 3}, {5, 7} as 16-bit pairs; the group's sum of x' and 2^-e.
+template <int MT>
+struct XChunk {
+  uint32_t w[MT][4][4];
+  int sx[MT];
+  float inv[MT];
+};
+
+template <int MT>
+__device__ __forceinline__ void load_x_raw(uint4 (&xr)[MT][4], const __nv_bfloat16* __restrict__ X,
+                                           int c, const Shape& sh, int lane) {
+  const int k = c * CHUNK + 32 * lane;
 #pragma unroll
-      for (int r = 0; r < R; ++r) cp_async16(dst + r * 32, src + r * rowb);
-    } else {
+  for (int m = 0; m < MT; ++m)
 #pragma unroll
-      for (int r = 0; r < R; ++r)
-        if (p.b * R + r < sh.N) cp_async16(dst + r * 32, src + r * rowb);
+    for (int q = 0; q < 4; ++q) {
+      xr[m][q] = make_uint4(0, 0, 0, 0);
+      if (m < sh.M && k < sh.K)
+        xr[m][q] = __ldg(reinterpret_cast<const uint4*>(X + size_t(m) * sh.K + k) + q);
     }
-  }
-  cp_async_commit();
 }
 
-// Scales (as fp32) and zero points (as integers) of one item for its R rows.
-struct ItemSZ {
-  float s[R];
-  int z[R];
-};
-
-// Loads v for the item at p when `live` (a lane past K, or a row past N,
-// keeps what it had: its values are never used).  Zero points are loaded only
-// for asymmetric weights; symmetric ones keep z = 8.
-__device__ __forceinline__ void load_sz(ItemSZ& v, const __half* __restrict__ scales,
-                                        const __half* __restrict__ zeros, Pos p, bool live,
-                                        const Shape& sh, int lane) {
-  const int k = p.c * CHUNK + lane * 32;
-  if (!live || k >= sh.K) return;
-  const size_t gi = size_t(p.b * R) * size_t(sh.G) + (k >> 7);
-  const __half* sp = scales + gi;
-  const __half* zp = zeros + gi;
-  if (p.b * R + R <= sh.N) {
+// Bring the lane's 64 bytes of a chunk of X into L1 ahead of its use.
+template <int MT>
+__device__ __forceinline__ void prefetch_x(const __nv_bfloat16* __restrict__ X, int c,
+                                           const Shape& sh, int lane) {
+  const int k = c * CHUNK + 32 * lane;
 #pragma unroll
-    for (int r = 0; r < R; ++r) v.s[r] = __half2float(__ldg(sp + r * sh.G));
-    if (!sh.sym) {
-#pragma unroll
-      for (int r = 0; r < R; ++r) v.z[r] = __half2int_rn(__ldg(zp + r * sh.G));
-    }
-  } else {
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-      if (p.b * R + r < sh.N) {
-        v.s[r] = __half2float(__ldg(sp + r * sh.G));
-        if (!sh.sym) v.z[r] = __half2int_rn(__ldg(zp + r * sh.G));
-      }
-  }
+  for (int m = 0; m < MT; ++m)
+    if (m < sh.M && k < sh.K)
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(X + size_t(m) * sh.K + k));
 }
 
 template <int MT>
-__device__ __forceinline__ void compute_item(const uint4* __restrict__ words, const ItemSZ& v,
-                                             float (&acc)[R][MT], const uint4* __restrict__ xs,
-                                             const int* __restrict__ sx,
-                                             const float* __restrict__ invs, int c,
-                                             const Shape& sh, int lane) {
-  const int k = c * CHUNK + lane * 32;
-  if (k >= sh.K) return;
-  const int g = k >> 7;
-  uint4 wr[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) wr[r] = words[r * 32];
-  int ah[R][MT], al[R][MT];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int m = 0; m < MT; ++m) ah[r][m] = al[r][m] = 0;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint32_t ev[R], od[R];  // even / odd elements of word q as bytes, per row
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const uint32_t w = q == 0 ? wr[r].x : q == 1 ? wr[r].y : q == 2 ? wr[r].z : wr[r].w;
-      ev[r] = w & 0x0F0F0F0Fu;
-      od[r] = (w >> 4) & 0x0F0F0F0Fu;
-    }
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      if (m < sh.M) {
-        const uint4 xq = xs[(m * sh.C + c) * 128 + q * 32 + lane];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          ah[r][m] = dp4a_us(ev[r], xq.x, ah[r][m]);
-          al[r][m] = dp4a_us(ev[r], xq.y, al[r][m]);
-          ah[r][m] = dp4a_us(od[r], xq.z, ah[r][m]);
-          al[r][m] = dp4a_us(od[r], xq.w, al[r][m]);
-        }
-      }
-    }
-  }
+__device__ __forceinline__ void convert_x(const uint4 (&xr)[MT][4], XChunk<MT>& xc) {
+  const float magic = __uint_as_float(MAGIC);
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
-    if (m < sh.M) {
-      const int sxl = sx[(m * sh.C + c) * 32 + lane];
-      const float fi = invs[m * sh.G + g];
+    uint32_t mx = 0;
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int t = ah[r][m] * 128 + al[r][m] - v.z[r] * sxl;  // exact
-        acc[r][m] = fmaf(float(t), v.s[r] * fi, acc[r][m]);
+    for (int q = 0; q < 4; ++q) {
+      mx = maxabs_bf16x2(mx, xr[m][q].x);
+      mx = maxabs_bf16x2(mx, xr[m][q].y);
+      mx = maxabs_bf16x2(mx, xr[m][q].z);
+      mx = maxabs_bf16x2(mx, xr[m][q].w);
+    }
+    // |x| bit patterns order like the values; the group is 4 lanes
+    uint32_t amax = max(mx & 0x7FFFu, (mx >> 16) & 0x7FFFu);
+    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    // amax in [2^(E-127), 2^(E-126)) for its biased exponent E; 2^e puts it
+    // in [2^12, 2^13).  A zero (or subnormal) group takes the largest step.
+    const int E = int(amax >> 7);
+    const int e = max(min(139 - E, 126), -126);
+    const float sc = __uint_as_float(uint32_t(127 + e) << 23);
+    uint32_t sum = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t wv[4] = {xr[m][q].x, xr[m][q].y, xr[m][q].z, xr[m][q].w};
+      uint32_t b[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        // fma rounds x * 2^e (exact) + 1.5 * 2^23 once, to the nearest
+        // integer (ties to even): the bit pattern is MAGIC + x'
+        b[2 * i] = __float_as_uint(fmaf(__uint_as_float(wv[i] << 16), sc, magic));
+        b[2 * i + 1] = __float_as_uint(fmaf(__uint_as_float(wv[i] & 0xFFFF0000u), sc, magic));
+        sum += b[2 * i] + b[2 * i + 1];
       }
+      xc.w[m][q][0] = prmt(b[0], b[2], 0x5410);  // x'0, x'2
+      xc.w[m][q][1] = prmt(b[4], b[6], 0x5410);  // x'4, x'6
+      xc.w[m][q][2] = prmt(b[1], b[3], 0x5410);  // x'1, x'3
+      xc.w[m][q][3] = prmt(b[5], b[7], 0x5410);  // x'5, x'7
+    }
+    int s = int(sum - 32u * MAGIC);  // the lane's sum of x' (mod 2^32, exact)
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    xc.sx[m] = s;
+    xc.inv[m] = __uint_as_float(uint32_t(127 - e) << 23);
+  }
+}
+
+// Scales and zero points of the 2 rows a lane finishes in an item: rows
+// 2 j, 2 j + 1 (j = lane & 3) of group lane / 4 of the chunk, kept as the
+// raw fp16 bits (converted only where they are used, so that the loads stay
+// in flight until then: no instruction may consume them at load time).  Rows outside the CTA's range and groups past K get
+// s = 0.
+struct SZ {
+  unsigned short s[2], z[2];
+};
+
+__device__ __forceinline__ void load_sz(SZ& v, const __half* __restrict__ scales,
+                                        const __half* __restrict__ zeros, Item p, bool live,
+                                        int row0, int row1, const Shape& sh, int lane) {
+  if (!live) return;
+  const int g = p.c * (CHUNK / 128) + (lane >> 2);
+  const int r = row0 + p.t * RB + 2 * (lane & 3);
+  const unsigned short* sp = reinterpret_cast<const unsigned short*>(scales);
+  const unsigned short* zp = reinterpret_cast<const unsigned short*>(zeros);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    v.s[k] = 0;       // +0.0
+    v.z[k] = 0x4800;  // 8.0: the symmetric code offset
+    if (r + k < row1 && g < sh.G) {
+      const size_t i = size_t(r + k) * sh.G + g;
+      v.s[k] = __ldg(sp + i);
+      if (!sh.sym) v.z[k] = __ldg(zp + i);
     }
   }
 }
 
-// The warp's sums for row block b: Y directly when the warp covered all of
-// it, else a partial in the warp's shared-memory slot (0: the warp's first
-// row block, 1: its last).
-template <int MT>
-__device__ __forceinline__ void emit_block(float (&acc)[R][MT], int b, bool whole, int slot,
-                                           float* __restrict__ part_w,
-                                           __nv_bfloat16* __restrict__ Y, const Shape& sh,
-                                           int lane) {
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      float v = acc[r][m];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      acc[r][m] = 0.f;
-      if (lane == 0) {
-        if (whole) {
-          if (m < sh.M && b * R + r < sh.N) Y[size_t(m) * sh.N + b * R + r] = __float2bfloat16_rn(v);
-        } else {
-          part_w[(slot * R + r) * MT_MAX + m] = v;
-        }
-      }
-    }
+// Issue the TMA loads of item p into a ring slot: one box of 4 rows x 512
+// bytes per 4 rows (the rows of a CTA come in multiples of 4; a chunk past K
+// reads zeros).  One lane issues them: a tensor copy takes warp-uniform
+// operands, so a single issuing lane needs no per-lane serialisation.
+__device__ __forceinline__ void issue_item(uint8_t* slot, uint64_t* bar, const CUtensorMap* tmap,
+                                           Item p, int row0, int row1, int lane) {
+  if (lane == 0) {
+    const int r0 = row0 + p.t * RB;
+    const int boxes = min(RB, row1 - r0) / 4;
+    tc::mbar_arrive_expect_tx(bar, uint32_t(boxes) * BOX_BYTES);
+    tc::tma_load_2d(slot, tmap, bar, p.c * (ROW_BYTES / 4), r0);
+    if (boxes > 1) tc::tma_load_2d(slot + BOX_BYTES, tmap, bar, p.c * (ROW_BYTES / 4), r0 + 4);
+  }
 }
 
-// Shared memory: [ring: 16 warps x D x R x 32 lanes x 16 B][X limbs: M C 128 x 16 B]
-//                [lane sums: M C 32 ints][2^-e: M G floats][partials: 16 x 2 x R x 2 floats]
-template <int MT, int D>
-__global__ void __launch_bounds__(THREADS, 1) gemv_cc_kernel(
-    const __nv_bfloat16* __restrict__ X, const uint8_t* __restrict__ codes,
-    const __half* __restrict__ scales, const __half* __restrict__ zeros,
-    __nv_bfloat16* __restrict__ Y, Shape sh) {
-  extern __shared__ uint4 smem[];
-  uint4* ring = smem;
-  uint4* xs = smem + WARPS * D * R * 32;
-  int* sx = reinterpret_cast<int*>(xs + sh.M * sh.C * 128);
-  float* invs = reinterpret_cast<float*>(sx + sh.M * sh.C * 32);
-  float* part = invs + sh.M * sh.G;
+// Bounded wait of the whole warp on a slot's mbarrier; false (and the error
+// recorded) when the deadline passed.
+__device__ __forceinline__ bool wait_slot(uint64_t* bar, uint32_t parity, uint64_t deadline,
+                                          int* status) {
+  bool ok = tc::mbar_try_wait(bar, parity);
+  uint32_t spins = 0;
+  while (!ok) {
+    ok = tc::mbar_try_wait(bar, parity);
+    if (!ok && (++spins & 31u) == 0 && tc::globaltimer_ns() > deadline) break;
+  }
+  const bool all = __all_sync(0xffffffffu, ok);
+  if (!all && (threadIdx.x & 31) == 0) record_error(status, WQ_ERR_TIMEOUT);
+  return all;
+}
+
+// Shared memory: [ring: W x D x ITEM_BYTES][mbarriers: W x D]
+//                [chunk partials: rows_max x C x MT floats]
+template <int MT, int D, int W>
+__global__ void __launch_bounds__(W * 32, (W <= 8 && MT <= 2) ? 2 : 1)
+    gemv_cc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __restrict__ X,
+                   const __half* __restrict__ scales, const __half* __restrict__ zeros,
+                   __nv_bfloat16* __restrict__ Y, Shape sh, int* status, uint64_t wait_ns) {
+  extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint4* ring_w = ring + warp * (D * R * 32);
+  uint8_t* ring_w = smem + size_t(warp) * D * ITEM_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(W) * D * ITEM_BYTES) + warp * D;
+  float* part = reinterpret_cast<float*>(smem + size_t(W) * D * ITEM_BYTES +
+                                         size_t(W) * D * sizeof(uint64_t));
 
-  // this CTA's row blocks and items; warp j takes items [s_j, s_{j+1})
-  const int rb0 = int((int64_t(blockIdx.x) * sh.NB) / gridDim.x);
-  const int rb1 = int((int64_t(blockIdx.x + 1) * sh.NB) / gridDim.x);
-  const int64_t ic = int64_t(rb1 - rb0) * sh.C;
-  const int64_t s0 = (ic * warp) / WARPS, s1 = (ic * (warp + 1)) / WARPS;
+  // this CTA's rows, row tiles and items; warp w takes items [s_w, s_{w+1})
+  const int row0 = 4 * int(int64_t(blockIdx.x) * sh.NB / gridDim.x);
+  const int row1 = min(4 * int(int64_t(blockIdx.x + 1) * sh.NB / gridDim.x), sh.N);
+  const int T = (row1 - row0 + RB - 1) / RB;
+  const int64_t I = int64_t(T) * sh.C;
+  const int64_t s0 = I * warp / W, s1 = I * (warp + 1) / W;
   const int n_it = int(s1 - s0);
-  Pos cur{rb0 + int(s0 / sh.C), int(s0 % sh.C)};
-  const int b_first = cur.b;
+  Item cur{int(s0 / T), int(s0 % T)};
 
-  // A kernel launched right after this one may be scheduled as soon as SMs
-  // free up; it only prefetches weights until this grid has finished.
+  if (lane == 0) {
+#pragma unroll
+    for (int d = 0; d < D; ++d) tc::mbar_init(bars + d, 1);
+    tc::fence_mbar_init();
+    tc::tma_prefetch_desc(&tmap);
+  }
+  __syncwarp();
+  // The next kernel on the stream may be scheduled as soon as SMs have room;
+  // it only prefetches weights until this grid has finished.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const uint64_t deadline = tc::globaltimer_ns() + wait_ns;
+
   // the warp's first D items go out before anything else
-  Pos ahead = cur;
+  Item ahead = cur;
 #pragma unroll
   for (int d = 0; d < D; ++d) {
-    issue_item(ring_w, d, codes, ahead, d < n_it, sh, lane);
-    ahead.next(sh.C);
+    if (d < n_it) issue_item(ring_w + d * ITEM_BYTES, bars + d, &tmap, ahead, row0, row1, lane);
+    ahead.next(T);
   }
   // scales and zero points run two items ahead, in two alternating sets
-  ItemSZ va, vb;
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    va.s[r] = vb.s[r] = 0.f;
-    va.z[r] = vb.z[r] = 8;
-  }
-  Pos szp = cur;
-  load_sz(va, scales, zeros, szp, 0 < n_it, sh, lane);
-  szp.next(sh.C);
-  load_sz(vb, scales, zeros, szp, 1 < n_it, sh, lane);
-  szp.next(sh.C);
+  SZ va, vb;
+  Item szp = cur;
+  load_sz(va, scales, zeros, szp, 0 < n_it, row0, row1, sh, lane);
+  szp.next(T);
+  load_sz(vb, scales, zeros, szp, 1 < n_it, row0, row1, sh, lane);
+  szp.next(T);
+
   // X may be the previous kernel's output, and Y its input: wait for that
   // grid (when launched as its dependent) before touching either
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  prepare_x(X, sh.M, sh.K, sh.C, xs, sx, invs);
-  __syncthreads();
 
-  float acc[R][MT];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
-  float* part_w = part + warp * (2 * R * MT_MAX);
+  XChunk<MT> xc;
+  int xchunk = -1;
   int slot = 0;
-  int c_start = cur.c;  // first chunk of the current row block this warp holds
-  // one item: compute it from the ring and `v`, refill its slot with the item
-  // D ahead, load `v` for the item two ahead, emit finished row blocks
-  auto step = [&](ItemSZ& v, int it) {
-    cp_async_wait<D - 1>();  // this lane's copies of item `it` have landed
-    compute_item<MT>(ring_w + slot * R * 32 + lane, v, acc, xs, sx, invs, cur.c, sh, lane);
-    // refill the slot just read (its words are in registers) with item it + D
-    issue_item(ring_w, slot, codes, ahead, it + D < n_it, sh, lane);
-    ahead.next(sh.C);
-    slot = (slot + 1 == D) ? 0 : slot + 1;
-    load_sz(v, scales, zeros, szp, it + 2 < n_it, sh, lane);
-    szp.next(sh.C);
-    if (cur.c == sh.C - 1 || it + 1 == n_it) {
-      emit_block<MT>(acc, cur.b, c_start == 0 && cur.c == sh.C - 1, cur.b == b_first ? 0 : 1,
-                     part_w, Y, sh, lane);
-      c_start = 0;
+  uint32_t parity = 0;
+  bool ok = true;
+  int done = 0;  // items whose slot wait has completed
+
+  auto step = [&](SZ& v, int it) {
+    if (cur.c != xchunk) {
+      uint4 xr[MT][4];
+      load_x_raw<MT>(xr, X, cur.c, sh, lane);
+      convert_x<MT>(xr, xc);
+      xchunk = cur.c;
     }
-    cur.next(sh.C);
+    Item nx = cur;
+    nx.next(T);
+    // the next chunk's X is brought into L1 one item before it is needed
+    if (it + 1 < n_it && nx.c != cur.c) prefetch_x<MT>(X, nx.c, sh, lane);
+
+    ok = wait_slot(bars + slot, parity, deadline, status);
+    if (!ok) return;
+    ++done;
+    const uint8_t* sb = ring_w + slot * ITEM_BYTES + lane * 16;
+    uint4 w4[RB];
+#pragma unroll
+    for (int r = 0; r < RB; ++r) w4[r] = lds128(sb + r * ROW_BYTES);
+    // The slot's codes are read (the warp barrier orders every lane's reads
+    // before the copies that overwrite them): refill it with the item D
+    // ahead before computing, so that D items per warp stay in flight.
+    __syncwarp();
+    if (it + D < n_it)
+      issue_item(ring_w + slot * ITEM_BYTES, bars + slot, &tmap, ahead, row0, row1, lane);
+    ahead.next(T);
+    if (++slot == D) {
+      slot = 0;
+      parity ^= 1u;
+    }
+
+    int tr[RB][MT];
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+      const uint32_t wv[4] = {w4[r].x, w4[r].y, w4[r].z, w4[r].w};
+      int ae[MT], ao[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) ae[m] = ao[m] = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t ev = wv[q] & 0x0F0F0F0Fu;  // u of elements 0, 2, 4, 6
+        const uint32_t od = wv[q] & 0xF0F0F0F0u;  // 16 u of elements 1, 3, 5, 7
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          ae[m] = dp2a_lo(xc.w[m][q][0], ev, ae[m]);
+          ae[m] = dp2a_hi(xc.w[m][q][1], ev, ae[m]);
+          ao[m] = dp2a_lo(xc.w[m][q][2], od, ao[m]);
+          ao[m] = dp2a_hi(xc.w[m][q][3], od, ao[m]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m) tr[r][m] = ae[m] + (ao[m] >> 4);  // exact
+    }
+
+    // 4 lanes of a group: lane j keeps rows 2 j, 2 j + 1 (exact integers)
+    const bool b1 = lane & 2, b0 = lane & 1, b2 = lane & 4;
+    int u4[4][MT];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const int keep = b1 ? tr[4 + k][m] : tr[k][m];
+        const int send = b1 ? tr[k][m] : tr[4 + k][m];
+        u4[k][m] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+      }
+    float p[2][MT];
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const int keep = b0 ? u4[2 + k][m] : u4[k][m];
+        const int send = b0 ? u4[k][m] : u4[2 + k][m];
+        const int zk = __half2int_rn(__ushort_as_half(v.z[k]));
+        const int t = keep + __shfl_xor_sync(0xffffffffu, send, 1) - zk * xc.sx[m];
+        p[k][m] = (float(t) * __half2float(__ushort_as_half(v.s[k]))) * xc.inv[m];
+      }
+    // the 8 groups of the chunk: lane keeps row 2 j + b2, then sums over b3, b4
+    float P[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const float keep = b2 ? p[1][m] : p[0][m];
+      const float send = b2 ? p[0][m] : p[1][m];
+      P[m] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+      P[m] += __shfl_xor_sync(0xffffffffu, P[m], 8);
+      P[m] += __shfl_xor_sync(0xffffffffu, P[m], 16);
+    }
+    if (lane < 8) {
+      const int rl = cur.t * RB + 4 * int(b1) + 2 * int(b0) + int(b2);  // row within the CTA
+      if (row0 + rl < row1) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) part[(size_t(rl) * sh.C + cur.c) * MT + m] = P[m];
+      }
+    }
+    load_sz(v, scales, zeros, szp, it + 2 < n_it, row0, row1, sh, lane);
+    szp.next(T);
+    cur = nx;
   };
-  for (int it = 0; it < n_it; it += 2) {
+  for (int it = 0; it < n_it && ok; it += 2) {
     step(va, it);
-    if (it + 1 == n_it) break;
+    if (it + 1 == n_it || !ok) break;
     step(vb, it + 1);
   }
-  cp_async_wait<0>();
+  if (!ok) {
+    // a copy did not land in time: wait (bounded) for the copies this warp
+    // still has in flight so that none lands after the kernel has exited
+    const uint64_t drain = tc::globaltimer_ns() + tc::kDrainNs;
+    for (int i = done; i < n_it && i < done + D; ++i) {
+      tc::wait_until(bars + slot, parity, drain);
+      if (++slot == D) {
+        slot = 0;
+        parity ^= 1u;
+      }
+    }
+  }
   __syncthreads();
 
-  // row blocks that straddle warp ranges: sum the partials in warp order
-  const int nbl = rb1 - rb0;
-  for (int t = threadIdx.x; t < nbl * R * MT; t += blockDim.x) {
-    const int bl = t / (R * MT), rm = t - bl * (R * MT), r = rm / MT, m = rm - r * MT;
-    const int64_t f = int64_t(bl) * sh.C, l = f + sh.C - 1;  // the block's first, last item
-    int jf = 0, jl = 0;
-    for (int j = 1; j < WARPS; ++j) {
-      const int64_t sj = (ic * j) / WARPS;
-      if (sj <= f) jf = j;
-      if (sj <= l) jl = j;
-    }
-    // jf..jl: warps whose ranges meet the block (empty ranges have no items
-    // and are skipped: their start equals the next warp's)
-    if (jf == jl) continue;  // one warp held all of it and wrote Y
-    float v = 0.f;
-    for (int j = jf; j <= jl; ++j) {
-      const int64_t sj = (ic * j) / WARPS, ej = (ic * (j + 1)) / WARPS;
-      if (sj == ej) continue;
-      const int sl = (rb0 + int(sj / sh.C) == rb0 + bl) ? 0 : 1;
-      v += part[j * (2 * R * MT_MAX) + (sl * R + r) * MT_MAX + m];
-    }
-    const int n = (rb0 + bl) * R + r;
-    if (m < sh.M && n < sh.N) Y[size_t(m) * sh.N + n] = __float2bfloat16_rn(v);
+  // a row's chunk partials, added in chunk order
+  const int nrows = row1 - row0;
+  for (int idx = threadIdx.x; idx < nrows * MT; idx += W * 32) {
+    const int r = idx / MT, m = idx - r * MT;
+    if (m >= sh.M) continue;
+    const float* pr = part + size_t(r) * sh.C * MT + m;
+    float acc = 0.f;
+    for (int c = 0; c < sh.C; ++c) acc += pr[size_t(c) * MT];
+    Y[size_t(m) * sh.N + row0 + r] = __float2bfloat16_rn(acc);
   }
 }
 
@@ -412,46 +448,83 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_cc_kernel(
 
 namespace wq_host {
 
-static int64_t cc_chunks(int64_t K) { return (K + wq::gemv_cc::CHUNK - 1) / wq::gemv_cc::CHUNK; }
+namespace {
 
-// Shared memory of the prepared X (limbs, lane sums, 2^-e factors) and of the
-// warps' partial sums.
-static size_t cc_x_smem(int64_t M, int64_t K) {
-  using namespace wq::gemv_cc;
-  const size_t C = size_t(cc_chunks(K));
-  return size_t(M) * C * CHUNK * 2 + size_t(M) * C * 32 * 4 + size_t(M) * size_t(K / 128) * 4 +
-         size_t(WARPS) * 2 * R * MT_MAX * 4;
+using namespace wq::gemv_cc;
+
+int cc_mt(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : 4; }
+
+Shape cc_shape(int64_t M, int64_t N, int64_t K, int sym, int P) {
+  Shape sh;
+  sh.M = int(M);
+  sh.N = int(N);
+  sh.K = int(K);
+  sh.G = int(K / 128);
+  sh.C = int((K + CHUNK - 1) / CHUNK);
+  sh.NB = int((N + 3) / 4);
+  sh.rows_max = 4 * int((int64_t(sh.NB) + P - 1) / P);
+  sh.sym = sym;
+  return sh;
 }
 
-int gemv_cc_depth(int64_t M, int64_t K) {
-  using namespace wq::gemv_cc;
-  if (M < 1 || M > kGemvCcMaxM) return 0;
-  const int64_t room = int64_t(SMEM_LIMIT) - int64_t(cc_x_smem(M, K));
-  const int64_t per_slot = int64_t(WARPS) * ITEM_BYTES;
-  const int64_t d = room > 0 ? room / per_slot : 0;
-  return d >= 2 ? int(d < MAXD ? d : MAXD) : 0;
+int cc_grid(int64_t N) {
+  const int64_t nb = (N + 3) / 4;
+  const int P = sm_count();
+  return int(nb < P ? nb : P);
 }
 
-template <int MT, int D>
-static cudaError_t launch_cc(dim3 grid, size_t smem, cudaStream_t s, const __nv_bfloat16* X,
-                             const uint8_t* codes, const __half* scales, const __half* zeros,
-                             __nv_bfloat16* Y, const wq::gemv_cc::Shape& sh) {
+size_t cc_smem(int mt, int D, int W, const Shape& sh) {
+  return size_t(W) * D * ITEM_BYTES + size_t(W) * D * sizeof(uint64_t) +
+         size_t(sh.rows_max) * size_t(sh.C) * size_t(mt) * sizeof(float);
+}
+
+// Launch shape.  Small matrices (N K <= 2^25): 8 warps with 3 ring slots
+// each (96 KB, at most 128 registers per thread at M <= 2), so that the next
+// decode kernel's CTA fits on the same SM and streams its first items under
+// the programmatic dependent launch -- on these shapes the fixed cost of a
+// launch dominates.  Larger ones: 12 warps with 2 slots each, which keeps
+// more items in compute at once and streams faster, at the price of
+// occupying the SM alone.  Measured on B200 at M = 1: 4096 x 4096 3.6 vs
+// 4.2 us, 11008 x 4096 7.4 vs 6.7 us, 28672 x 8192 32 vs 23.5 us.
+struct CcConfig {
+  int W, D;
+};
+
+CcConfig cc_config(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || M > kGemvCcMaxM || N < 1 || K < 128) return {0, 0};
+  const Shape sh = cc_shape(M, N, K, 1, cc_grid(N));
+  const CcConfig pref = N * K <= (int64_t(1) << 25) ? CcConfig{8, 3} : CcConfig{12, 2};
+  const CcConfig tries[3] = {pref, {8, 2}, {0, 0}};
+  for (const CcConfig& c : tries)
+    if (c.W > 0 && cc_smem(cc_mt(M), c.D, c.W, sh) <= size_t(SMEM_LIMIT)) return c;
+  return {0, 0};
+}
+
+std::mutex g_cc_attr_mu;
+
+template <int MT, int D, int W>
+cudaError_t launch_cc(int grid, size_t smem, cudaStream_t s, const CUtensorMap& tmap,
+                      const __nv_bfloat16* X, const __half* scales, const __half* zeros,
+                      __nv_bfloat16* Y, const Shape& sh) {
   static bool attr_done[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 64 && !attr_done[dev]) {
-    e = cudaFuncSetAttribute(wq::gemv_cc::gemv_cc_kernel<MT, D>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             wq::gemv_cc::SMEM_LIMIT);
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(g_cc_attr_mu);
+    if (!attr_done[dev]) {
+      e = cudaFuncSetAttribute(gemv_cc_kernel<MT, D, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SMEM_LIMIT);
+      if (e != cudaSuccess) return e;
+      attr_done[dev] = true;
+    }
   }
   // programmatic dependent launch: the weight prefetch of this kernel
   // overlaps the tail of the kernel before it on the stream
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(wq::gemv_cc::THREADS);
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(W * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -459,40 +532,40 @@ static cudaError_t launch_cc(dim3 grid, size_t smem, cudaStream_t s, const __nv_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, wq::gemv_cc::gemv_cc_kernel<MT, D>, X, codes, scales, zeros, Y,
-                            sh);
+  return cudaLaunchKernelEx(&cfg, gemv_cc_kernel<MT, D, W>, tmap, X, scales, zeros, Y, sh,
+                            status_ptr(), wait_limit_ns());
 }
+
+}  // namespace
+
+bool gemv_cc_fits(int64_t M, int64_t N, int64_t K) { return cc_config(M, N, K).W > 0; }
 
 int launch_gemv_w4a16_cc(const void* X, int64_t M, int64_t K, const void* codes,
                          const void* scales, const void* zeros, int64_t N, int sym, void* Y,
                          cudaStream_t s) {
-  using namespace wq::gemv_cc;
-  const int D = gemv_cc_depth(M, K);
-  if (D == 0) return WQ_ERR_ARG;
-  Shape sh;
-  sh.M = int(M);
-  sh.N = int(N);
-  sh.K = int(K);
-  sh.G = int(K / 128);
-  sh.C = int(cc_chunks(K));
-  sh.NB = int((N + R - 1) / R);
-  sh.sym = sym;
-  const int P = sm_count();
-  const dim3 grid(unsigned(sh.NB < P ? sh.NB : P));
-  const size_t smem = size_t(WARPS) * D * ITEM_BYTES + cc_x_smem(M, K);
+  const CcConfig cf = cc_config(M, N, K);
+  if (cf.W == 0) return WQ_ERR_ARG;
+  const int grid = cc_grid(N);
+  const Shape sh = cc_shape(M, N, K, sym, grid);
+  const int mt = cc_mt(M);
+  const size_t smem = cc_smem(mt, cf.D, cf.W, sh);
 
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(X);
   const __half* sc = static_cast<const __half*>(scales);
   const __half* zp = static_cast<const __half*>(zeros);
-  const uint8_t* cd = static_cast<const uint8_t*>(codes);
   __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y);
+  // the codes as rows of K / 8 32-bit words; a box is 4 rows x 128 words
+  CUtensorMap tmap;
+  const int st = make_tmap_2d(&tmap, codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(N),
+                              uint64_t(K / 8), 4, ROW_BYTES / 4, 0);
+  if (st != WQ_OK) return st;
   cudaError_t e = cudaErrorInvalidValue;
-  const int mt = M <= 1 ? 1 : M <= 2 ? 2 : 4;  // M = 3 runs the 4-row instance
-#define WQ_CC_CASE(MT_, D_) \
-  if (mt == MT_ && D == D_) e = launch_cc<MT_, D_>(grid, smem, s, x, cd, sc, zp, y, sh);
-  WQ_CC_CASE(1, 2) WQ_CC_CASE(1, 3) WQ_CC_CASE(1, 4) WQ_CC_CASE(1, 5) WQ_CC_CASE(1, 6)
-  WQ_CC_CASE(2, 2) WQ_CC_CASE(2, 3) WQ_CC_CASE(2, 4) WQ_CC_CASE(2, 5) WQ_CC_CASE(2, 6)
-  WQ_CC_CASE(4, 2) WQ_CC_CASE(4, 3) WQ_CC_CASE(4, 4) WQ_CC_CASE(4, 5) WQ_CC_CASE(4, 6)
+#define WQ_CC_CASE(MT_, D_, W_)                   \
+  if (mt == MT_ && cf.D == D_ && cf.W == W_) \
+    e = launch_cc<MT_, D_, W_>(grid, smem, s, tmap, x, sc, zp, y, sh);
+  WQ_CC_CASE(1, 3, 8) WQ_CC_CASE(1, 2, 8) WQ_CC_CASE(1, 2, 12)
+  WQ_CC_CASE(2, 3, 8) WQ_CC_CASE(2, 2, 8) WQ_CC_CASE(2, 2, 12)
+  WQ_CC_CASE(4, 3, 8) WQ_CC_CASE(4, 2, 8) WQ_CC_CASE(4, 2, 12)
 #undef WQ_CC_CASE
   if (e != cudaSuccess) return cuda_fail(e, "gemv_cc_kernel");
   return WQ_OK;

@@ -37,14 +37,14 @@ int launch_dequant_int4(const void* codes, const void* scales, const void* zeros
 int launch_dequant_int8_rows(const void* q, const void* scales, int64_t N, int64_t K, void* out,
                              int out_dtype, cudaStream_t s);
 
-// Decode products (M <= 16): the CUDA-core kernel (no workspace) for M <= 2,
-// and for M <= kGemvCcMaxM on small matrices, when its prepared X fits in
-// shared memory (gemv_cc_depth > 0); the tensor-core kernel otherwise.  The decode workspace holds
-// the tensor-core kernel's tile counters (zeroed by the caller once, left
-// zeroed by every completed call) and then its tile partials; it has the same
-// size for every M.
+// Decode products (M <= 16): the CUDA-core kernel (no workspace) for M <=
+// kGemvCcMaxM when its ring and row partials fit in shared memory
+// (gemv_cc_fits), the tensor-core kernel otherwise.  The decode workspace
+// holds the tensor-core kernel's tile counters (zeroed by the caller once,
+// left zeroed by every completed call) and then its tile partials; it has the
+// same size for every M.
 constexpr int64_t kGemvCcMaxM = 4;
-int gemv_cc_depth(int64_t M, int64_t K);
+bool gemv_cc_fits(int64_t M, int64_t N, int64_t K);
 int launch_gemv_w4a16_cc(const void* X, int64_t M, int64_t K, const void* codes,
                          const void* scales, const void* zeros, int64_t N, int sym, void* Y,
                          cudaStream_t s);

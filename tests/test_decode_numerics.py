@@ -1,9 +1,11 @@
 """Host restatement of the CUDA-core decode kernel's arithmetic (W4A16,
 M <= 4): each (activation row, 128-group) of X becomes integers
-x' = rint(x 2^e) with the group's max |x'| in [2^12, 2^13), split into int8
-limbs x' = 128 h + l; the group's dot product with the codes is an exact
-integer, scaled once by s 2^-e.  These tests pin the limb ranges DP4A needs,
-the exactness of the integer sums and the error bound against the fp64
+x' = rint(x 2^e) with the group's max |x'| in [2^12, 2^13), which fit the
+signed 16-bit halves of DP2A.  A code word's even nibbles (w & 0x0F0F0F0F)
+and sixteen times its odd ones (w & 0xF0F0F0F0) are taken against them in two
+integer sums per row and lane; the group's dot product is an exact integer,
+scaled once by s 2^-e.  These tests pin the operand ranges DP2A needs, the
+exactness and size of the integer sums and the error bound against the fp64
 product."""
 import numpy as np
 import pytest
@@ -22,7 +24,15 @@ def prepare(x):
     return xi, e
 
 
-def test_limbs_fit_dp4a():
+def magic_round(x, e):
+    """fma(x, 2^e, 1.5 2^23) in binary32, as the kernel computes x': the bit
+    pattern minus that of 1.5 2^23."""
+    prod = (x.astype(np.float64) * np.exp2(e)[:, None]).astype(np.float32)   # exact (power of 2)
+    r = (prod + np.float32(12582912.0)).astype(np.float32)                    # one rounding, RNE
+    return r.view(np.uint32).astype(np.int64) - 0x4B400000
+
+
+def test_operands_fit_dp2a():
     rng = np.random.default_rng(0)
     for scale in (1e-6, 1e-2, 1.0, 50.0, 3e4):
         x = oracle.bf16_to_f32(oracle.f32_to_bf16(
@@ -30,22 +40,34 @@ def test_limbs_fit_dp4a():
         xi, e = prepare(x)
         m = np.abs(xi).max(axis=1)
         assert ((m >= 2 ** 12) & (m <= 2 ** 13)).all()   # the rounded max may reach 2^13
-        h, l = xi >> 7, xi & 127
-        assert np.array_equal(128 * h + l, xi)
-        assert h.min() >= -64 and h.max() <= 64 and l.min() >= 0 and l.max() <= 127
+        assert xi.min() >= -2 ** 15 and xi.max() < 2 ** 15   # signed 16-bit halves
+        # the fma with 1.5 2^23 rounds to the same integers (ties to even)
+        assert np.array_equal(magic_round(x, e), xi)
+        # its low 16 bits are x' as a two's-complement 16-bit value
+        lo = (magic_round(x, e) + 0x4B400000) & 0xFFFF
+        assert np.array_equal(np.where(lo >= 2 ** 15, lo - 2 ** 16, lo), xi)
 
 
 def test_integer_sums_are_exact_and_small():
     rng = np.random.default_rng(1)
     x = oracle.bf16_to_f32(oracle.f32_to_bf16(rng.standard_normal((200, 128)).astype(np.float32))).reshape(200, 128)
     xi, _ = prepare(x)
+    # extreme operands: every code 15 against the largest |x'| everywhere
     u = rng.integers(0, 16, (200, 128))
     z = rng.integers(0, 16, (200, 1))
-    h, l = xi >> 7, xi & 127
-    per_lane = 128 * (u[:, :32] * h[:, :32]).sum(1) + (u[:, :32] * l[:, :32]).sum(1)
-    assert np.abs(per_lane).max() < 2 ** 22     # one lane's 32 elements: exact in int32 and fp32
-    t = 128 * (u * h).sum(1) + (u * l).sum(1) - z[:, 0] * xi.sum(1)
+    worst_even = 16 * 15 * 2 ** 13          # one lane: 16 even elements
+    worst_odd = 16 * (16 * 15) * 2 ** 13    # 16 odd elements, codes x 16
+    assert worst_even < 2 ** 31 and worst_odd < 2 ** 31
+    ev = (u[:, 0:32:2] * xi[:, 0:32:2]).sum(1)
+    od16 = ((16 * u[:, 1:32:2]) * xi[:, 1:32:2]).sum(1)
+    assert (od16 % 16 == 0).all()            # the odd sum divides exactly by 16
+    lane = ev + od16 // 16
+    assert np.array_equal(lane, (u[:, :32] * xi[:, :32]).sum(1))
+    # the group's sum minus the zero point's share is exact below 2^24, so
+    # its conversion to binary32 is exact too
+    t = (u * xi).sum(1) - z[:, 0] * xi.sum(1)
     assert np.array_equal(t, ((u - z) * xi).sum(1))
+    assert 15 * 128 * 2 ** 13 < 2 ** 24
 
 
 @pytest.mark.parametrize("sym", [True, False])
