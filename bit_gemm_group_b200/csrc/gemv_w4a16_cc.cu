@@ -10,7 +10,8 @@
 //
 // At M <= 4 there is too little arithmetic per weight byte for the tensor
 // cores to help: the kernel is a stream, and what bounds it is how many issue
-// slots it spends per byte and how many bytes it keeps in flight.
+// slots it spends per byte and how many bytes it keeps in flight (from M = 5
+// on, the multiply-adds go to the tensor cores: gemv_w4a16_mma.cu).
 //
 // Exact integer inner products.  X is rewritten per (activation row m,
 // group g of 128 along K) as integers x' = rint(x * 2^e), e chosen so that
@@ -452,7 +453,7 @@ namespace {
 
 using namespace wq::gemv_cc;
 
-int cc_mt(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : 4; }
+int cc_mt(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : 4; }  // M = 3 runs the 4-row instance
 
 Shape cc_shape(int64_t M, int64_t N, int64_t K, int sym, int P) {
   Shape sh;
@@ -502,24 +503,30 @@ CcConfig cc_config(int64_t M, int64_t N, int64_t K) {
 
 std::mutex g_cc_attr_mu;
 
+// the kernel's dynamic shared memory limit, once per device
 template <int MT, int D, int W>
-cudaError_t launch_cc(int grid, size_t smem, cudaStream_t s, const CUtensorMap& tmap,
-                      const __nv_bfloat16* X, const __half* scales, const __half* zeros,
-                      __nv_bfloat16* Y, const Shape& sh) {
-  static bool attr_done[64] = {};
+cudaError_t cc_attr() {
+  static bool done[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64) return cudaErrorInvalidDevice;
-  {
-    std::lock_guard<std::mutex> lock(g_cc_attr_mu);
-    if (!attr_done[dev]) {
-      e = cudaFuncSetAttribute(gemv_cc_kernel<MT, D, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SMEM_LIMIT);
-      if (e != cudaSuccess) return e;
-      attr_done[dev] = true;
-    }
+  std::lock_guard<std::mutex> lock(g_cc_attr_mu);
+  if (!done[dev]) {
+    e = cudaFuncSetAttribute(gemv_cc_kernel<MT, D, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_LIMIT);
+    if (e != cudaSuccess) return e;
+    done[dev] = true;
   }
+  return cudaSuccess;
+}
+
+template <int MT, int D, int W>
+cudaError_t launch_cc(int grid, size_t smem, cudaStream_t s, const CUtensorMap& tmap,
+                      const __nv_bfloat16* X, const __half* scales, const __half* zeros,
+                      __nv_bfloat16* Y, const Shape& sh) {
+  cudaError_t e = cc_attr<MT, D, W>();
+  if (e != cudaSuccess) return e;
   // programmatic dependent launch: the weight prefetch of this kernel
   // overlaps the tail of the kernel before it on the stream
   cudaLaunchConfig_t cfg = {};
@@ -539,6 +546,15 @@ cudaError_t launch_cc(int grid, size_t smem, cudaStream_t s, const CUtensorMap& 
 }  // namespace
 
 bool gemv_cc_fits(int64_t M, int64_t N, int64_t K) { return cc_config(M, N, K).W > 0; }
+
+int prepare_cc_kernels() {
+  const cudaError_t es[9] = {cc_attr<1, 3, 8>(), cc_attr<1, 2, 8>(), cc_attr<1, 2, 12>(),
+                             cc_attr<2, 3, 8>(), cc_attr<2, 2, 8>(), cc_attr<2, 2, 12>(),
+                             cc_attr<4, 3, 8>(), cc_attr<4, 2, 8>(), cc_attr<4, 2, 12>()};
+  for (cudaError_t e : es)
+    if (e != cudaSuccess) return cuda_fail(e, "gemv_cc_kernel attributes");
+  return WQ_OK;
+}
 
 int launch_gemv_w4a16_cc(const void* X, int64_t M, int64_t K, const void* codes,
                          const void* scales, const void* zeros, int64_t N, int sym, void* Y,

@@ -32,9 +32,11 @@ constexpr int THREADS = 256;
 constexpr int LPR = THREADS / RB;  // 8 lanes per row
 constexpr int CPT = GS / LPR;      // 16 columns per thread in the block update
 
-// Shared memory: U block [128][128] (128 KB), E block [32][128] (32 KB),
-// corrected weights [32][128] (32 KB).
-constexpr size_t SMEM_BYTES = size_t(GS) * GS * 8 + size_t(RB) * GS * 8 * 2;
+// Shared memory: U block [128][129] (rows padded by one double so that the
+// eight lanes of a row, reading entries 128 rows apart, hit distinct banks),
+// E block [32][129], corrected weights [32][129].
+constexpr int LD = GS + 1;
+constexpr size_t SMEM_BYTES = size_t(GS) * LD * 8 + size_t(RB) * LD * 8 * 2;
 
 // The round-to-nearest group rules on binary32 values (sym: s = amax / 7;
 // asym: s = (max - min) / 15, z = clamp(round(-min / s), 0, 15); the scale
@@ -68,9 +70,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint8_t* __restrict__ codes, __half* __restrict__ scales,
                 __half* __restrict__ zeros, double* __restrict__ err, int* status) {
   extern __shared__ double smem[];
-  double* Us = smem;                  // [GS][GS]
-  double* Es = Us + GS * GS;          // [RB][GS]
-  double* Ws = Es + RB * GS;          // [RB][GS]
+  double* Us = smem;                  // [GS][LD]
+  double* Es = Us + GS * LD;          // [RB][LD]
+  double* Ws = Es + RB * LD;          // [RB][LD]
   const int t = threadIdx.x;
   const int r = t / LPR, l8 = t % LPR;  // row within the CTA, lane within the row
   const int n = blockIdx.x * RB + r;
@@ -89,21 +91,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncthreads();
       for (int i = t; i < GS * GS / 2; i += THREADS) {   // U[p block, g block], 16-byte loads
         const int a = i / (GS / 2), b = (i % (GS / 2)) * 2;
-        reinterpret_cast<double2*>(Us)[i] =
-            *reinterpret_cast<const double2*>(U + size_t(p * GS + a) * K + j0 + b);
+        const double2 v = *reinterpret_cast<const double2*>(U + size_t(p * GS + a) * K + j0 + b);
+        Us[a * LD + b] = v.x;
+        Us[a * LD + b + 1] = v.y;
       }
       for (int i = t; i < RB * GS / 2; i += THREADS) {   // err[rows, p block]
         const int a = i / (GS / 2), b = (i % (GS / 2)) * 2;
         const int na = blockIdx.x * RB + a;
         double2 v = make_double2(0.0, 0.0);
         if (na < N) v = *reinterpret_cast<const double2*>(err + size_t(na) * K + p * GS + b);
-        reinterpret_cast<double2*>(Es)[i] = v;
+        Es[a * LD + b] = v.x;
+        Es[a * LD + b + 1] = v.y;
       }
       __syncthreads();
       for (int i = 0; i < GS; ++i) {
-        const double e = Es[r * GS + i];
+        const double e = Es[r * LD + i];
 #pragma unroll
-        for (int q = 0; q < CPT; ++q) c[q] = fma(e, Us[i * GS + l8 + LPR * q], c[q]);
+        for (int q = 0; q < CPT; ++q) c[q] = fma(e, Us[i * LD + l8 + LPR * q], c[q]);
       }
     }
     // ---- corrected group values and the group's parameters
@@ -113,7 +117,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int j = l8 + LPR * q;
       const double w0 = row_in ? double(to_f32<T>(W[size_t(n) * K + j0 + j])) : 0.0;
       const double wv = w0 - c[q];
-      Ws[r * GS + j] = wv;
+      Ws[r * LD + j] = wv;
       const float f = float(wv);
       bad |= !isfinite(f);
       amax = fmaxf(amax, fabsf(f));
@@ -141,18 +145,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();  // every warp is done with Us / Es of the block update
     for (int i = t; i < GS * GS / 2; i += THREADS) {     // U diagonal block
       const int a = i / (GS / 2), b = (i % (GS / 2)) * 2;
-      reinterpret_cast<double2*>(Us)[i] =
-          *reinterpret_cast<const double2*>(U + size_t(j0 + a) * K + j0 + b);
+      const double2 v = *reinterpret_cast<const double2*>(U + size_t(j0 + a) * K + j0 + b);
+      Us[a * LD + b] = v.x;
+      Us[a * LD + b + 1] = v.y;
     }
     __syncthreads();
     uint32_t packed = 0;  // the row's first lane assembles 8 nibbles per word
     for (int j = 0; j < GS; ++j) {
       double part = 0.0;
-      for (int i = l8; i < j; i += LPR) part = fma(Es[r * GS + i], Us[i * GS + j], part);
+      for (int i = l8; i < j; i += LPR) part = fma(Es[r * LD + i], Us[i * LD + j], part);
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
       if (l8 == 0) {
-        const double w = Ws[r * GS + j] - part;
+        const double w = Ws[r * LD + j] - part;
         int q = 0;
         double w_hat = 0.0;
         if (!degenerate) {
@@ -161,7 +166,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           q = min(max(int(rr) + z, qmin), qmax);
           w_hat = double(sf) * double(q - (sym ? 0 : z));
         }
-        Es[r * GS + j] = (w - w_hat) / Us[j * GS + j];
+        Es[r * LD + j] = (w - w_hat) / Us[j * LD + j];
         packed |= uint32_t(q - qmin) << (4 * (j & 7));
         if ((j & 7) == 7) {
           if (row_in)
@@ -173,7 +178,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     // this group's errors, for the block updates of the later groups
     if (row_in)
-      for (int j = l8; j < GS; j += LPR) err[size_t(n) * K + j0 + j] = Es[r * GS + j];
+      for (int j = l8; j < GS; j += LPR) err[size_t(n) * K + j0 + j] = Es[r * LD + j];
     __syncthreads();
   }
   if (bad) record_error(status, WQ_ERR_NONFINITE);

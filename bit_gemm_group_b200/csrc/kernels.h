@@ -57,6 +57,11 @@ bool decode_on_cuda_cores(int64_t M, int64_t N, int64_t K);
 int launch_decode_w4a16(const void* X, int64_t M, int64_t K, const void* codes,
                         const void* scales, const void* zeros, int64_t N, int sym, void* Y,
                         void* ws, cudaStream_t s);
+// Set the decode kernels' launch attributes on the current device (done
+// lazily by the launchers otherwise); WQ_OK or an error status.
+int prepare_decode_kernels();
+int prepare_cc_kernels();
+int prepare_tc_kernels();
 int launch_gemm_w4a16(const void* X, int64_t M, int64_t K, const void* codes,
                       const void* scales, const void* zeros, int64_t N, int sym, void* Y,
                       cudaStream_t s);

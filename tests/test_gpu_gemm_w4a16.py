@@ -57,7 +57,9 @@ def test_prefill_workload_sampled():
     dq, oq = quantized(W, True)
     X = wl.activation(2048, 4096)
     N = W.shape[0]
-    check(X, dq, oq, True, [(0, 256), (N - 384, N)])
+    # five 256/384-column windows spread over N, at the row-normalised bound
+    check(X, dq, oq, True, [(0, 256), (N // 4 - 128, N // 4 + 128), (N // 2 - 128, N // 2 + 128),
+                            (3 * N // 4 - 128, 3 * N // 4 + 128), (N - 384, N)])
     check(X[:64], dq, oq, True, [(1000, 1128)], elementwise=True)
 
 

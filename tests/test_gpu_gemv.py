@@ -76,6 +76,22 @@ def test_ragged(M, N, K, sym):
     check_gemv(make_activation(M, K, seed=M), dq, oq, sym, rounding_aware=N < 256)
 
 
+@pytest.mark.parametrize("M", [1, 4, 16])
+@pytest.mark.parametrize("N,K", [(8, 1152), (24, 1152), (136, 4096)])
+@pytest.mark.parametrize("sym", [True, False])
+def test_small_n_with_outlier_activations(M, N, K, sym):
+    """Few outputs per row and six activation dims of magnitude 50-100: the
+    CUDA-core kernel rounds each group's activations to 13-bit integers
+    relative to the group maximum, so a group that holds an outlier dim
+    rounds nearly all its other elements; with small N one output carries
+    much of the row norm.  The row-normalised bound (less the bf16 output
+    half-ulp) still holds."""
+    W = make_weight(N, K, 0.02, seed=N + 7 * K, outlier_frac=0.01, outlier_scale=30.0)
+    dq, oq = quantized(W, sym)
+    X = make_activation(M, K, seed=M + 31, outlier_dims=6)
+    check_gemv(X, dq, oq, sym, rounding_aware=True)
+
+
 @pytest.mark.parametrize("kind", ["positive", "outlier_dims", "row_scales", "sparse_groups"])
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_activation_structure(kind, M):
