@@ -517,6 +517,160 @@ __global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Per-row quantizers with the row held in registers (16-bit inputs, K in
+// {1024, 2048, 4096, 8192}): the activation side of W8A8 / FP8
+// ---------------------------------------------------------------------------
+// A row is K / 32 threads x 32 elements: thread t owns the 8-element blocks
+// t + (K / 256) i, i = 0..3 (each load and store instruction of a warp covers
+// contiguous bytes).  The row is read once; its maximum |x| is an integer max
+// over the 16-bit magnitude bit patterns (which order like the values; a NaN
+// or infinity pattern is at least the infinity pattern, so the same max
+// reports non-finite input), a warp shuffle tree and one barrier.  The codes
+// come from the same reciprocal-multiply rules as the two-pass kernels, so
+// they are identical.  KIND 0: int8 per token (s = max(amax / 127, 1e-8),
+// q in [-128, 127], optional SmoothQuant division by s[k]); KIND 1: E4M3
+// (s = max(amax / 448, 1e-8)).
+template <typename T>
+__device__ __forceinline__ uint32_t abs_bits_mask() {
+  return 0x7FFF7FFFu;
+}
+template <typename T>
+__device__ __forceinline__ uint32_t inf_bits();
+template <>
+__device__ __forceinline__ uint32_t inf_bits<__nv_bfloat16>() { return 0x7F80u; }
+template <>
+__device__ __forceinline__ uint32_t inf_bits<__half>() { return 0x7C00u; }
+
+template <typename T>
+__device__ __forceinline__ float half_bits_to_f32(uint32_t h);
+template <>
+__device__ __forceinline__ float half_bits_to_f32<__nv_bfloat16>(uint32_t h) {
+  return __uint_as_float(h << 16);
+}
+template <>
+__device__ __forceinline__ float half_bits_to_f32<__half>(uint32_t h) {
+  return __half2float(__ushort_as_half((unsigned short)h));
+}
+
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+template <typename T, int KIND>
+__global__ void __launch_bounds__(256) quantize_rows_reg_kernel(
+    const T* __restrict__ X, int64_t rows, int K, const float* __restrict__ smooth,
+    uint8_t* __restrict__ q, float* __restrict__ scales, int* status) {
+  __shared__ float red[8];
+  __shared__ int bad_w[8];
+  const int tpr = K >> 5;  // threads per row (a multiple of 32)
+  const int rpb = 256 / tpr;
+  const int wpr = tpr >> 5;
+  const int sub = threadIdx.x / tpr, t = threadIdx.x - sub * tpr;
+  const int warp = threadIdx.x >> 5;
+  for (int64_t r0 = int64_t(blockIdx.x) * rpb; r0 < rows; r0 += int64_t(gridDim.x) * rpb) {
+    const int64_t r = r0 + sub;
+    const bool live = r < rows;
+    const T* row = X + (live ? r : 0) * int64_t(K);
+    uint4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[i] = make_uint4(0, 0, 0, 0);
+      if (live) v[i] = __ldcs(reinterpret_cast<const uint4*>(row) + t + tpr * i);
+    }
+    float x[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        x[8 * i + 2 * j] = half_bits_to_f32<T>(w[j] & 0xFFFFu);
+        x[8 * i + 2 * j + 1] = half_bits_to_f32<T>(w[j] >> 16);
+      }
+    }
+    float amax = 0.f;
+    bool finite = true;
+    if (KIND == 0 && smooth != nullptr) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t k = 8 * int64_t(t + tpr * i);
+        const float4 a = *reinterpret_cast<const float4*>(smooth + k);
+        const float4 b = *reinterpret_cast<const float4*>(smooth + k + 4);
+        const float sv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          x[8 * i + e] = div_rn(x[8 * i + e], sv[e]);
+          finite &= isfinite(x[8 * i + e]);
+          amax = fmaxf(amax, fabsf(x[8 * i + e]));
+        }
+      }
+    } else {
+      uint32_t m = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        m = vmax_u16x2(m, v[i].x & abs_bits_mask<T>());
+        m = vmax_u16x2(m, v[i].y & abs_bits_mask<T>());
+        m = vmax_u16x2(m, v[i].z & abs_bits_mask<T>());
+        m = vmax_u16x2(m, v[i].w & abs_bits_mask<T>());
+      }
+      const uint32_t mb = max(m & 0xFFFFu, m >> 16);
+      finite = mb < inf_bits<T>();
+      if (finite) {
+        amax = half_bits_to_f32<T>(mb);
+      } else {
+        // non-finite input (reported): the maximum as the two-pass kernels
+        // take it, NaN ignored and infinity counted
+#pragma unroll
+        for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(x[e]));
+      }
+    }
+    amax = warp_max(amax);
+    const bool wbad = __any_sync(0xffffffffu, !finite);
+    if ((threadIdx.x & 31) == 0) {
+      red[warp] = amax;
+      bad_w[warp] = wbad;
+    }
+    __syncthreads();
+    int bad = 0;
+#pragma unroll 1
+    for (int j = 0; j < wpr; ++j) {
+      amax = fmaxf(amax, red[sub * wpr + j]);
+      bad |= bad_w[sub * wpr + j];
+    }
+    const float s = fmaxf(div_rn(amax, KIND == 0 ? 127.f : 448.f), 1e-8f);
+    const float inv = rcp_approx(s);
+    if (live && t == 0) {
+      scales[r] = s;
+      if (bad) record_error(status, WQ_ERR_NONFINITE);
+    }
+    if (live) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        union {
+          uint2 v2;
+          uint8_t b[8];
+        } o;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (KIND == 0) {
+            float rr = rint_quot_i8(x[8 * i + e], s, inv);
+            rr = fmaxf(-200.f, fminf(200.f, rr));
+            o.b[e] = uint8_t(int8_t(min(max(int(rr), -128), 127)));
+          } else {
+            o.b[e] = uint8_t(__nv_cvt_float_to_fp8(quot_e4m3(x[8 * i + e], s, inv),
+                                                   __NV_SATFINITE, __NV_E4M3));
+          }
+        }
+        *reinterpret_cast<uint2*>(q + r * int64_t(K) + 8 * int64_t(t + tpr * i)) = o.v2;
+      }
+    }
+    __syncthreads();  // red[] is reused by the next rows
+  }
+}
+
 // ---------------------------------------------------------------------------
 // SmoothQuant statistics ("27届大模型面试准备（十九）…" sec. 4.2)
 // ---------------------------------------------------------------------------
@@ -867,8 +1021,36 @@ int launch_quantize_int4(const void* W, int w_dtype, int64_t N, int64_t K, int g
   return WQ_ERR_ARG;
 }
 
+// The register-resident kernel serves 16-bit rows of K = 1024, 2048, 4096 or
+// 8192 elements: a row is K / 32 threads of 32 elements, and the 256-thread
+// block holds a whole number of rows.
+static bool rows_in_registers(int w_dtype, int64_t K) {
+  return (w_dtype == WQ_BF16 || w_dtype == WQ_F16) &&
+         (K == 1024 || K == 2048 || K == 4096 || K == 8192);
+}
+
+template <typename T, int KIND>
+static void launch_rows_reg(const void* W, int64_t N, int64_t K, const float* smooth, void* q,
+                            void* scales, cudaStream_t s) {
+  const int64_t rpb = 8192 / K;
+  const int64_t blocks = (N + rpb - 1) / rpb;
+  const int64_t cap = int64_t(sm_count()) * 8;
+  const int grid = int(blocks < cap ? blocks : cap);
+  wq::quantize_rows_reg_kernel<T, KIND><<<grid, 256, 0, s>>>(
+      static_cast<const T*>(W), N, int(K), smooth, static_cast<uint8_t*>(q),
+      static_cast<float*>(scales), status_ptr());
+}
+
 int launch_quantize_rows_i8(const void* W, int w_dtype, int64_t N, int64_t K, bool activation,
                             const float* smooth, void* q, void* scales, cudaStream_t s) {
+  if (activation && rows_in_registers(w_dtype, K)) {
+    if (w_dtype == WQ_BF16)
+      launch_rows_reg<__nv_bfloat16, 0>(W, N, K, smooth, q, scales, s);
+    else
+      launch_rows_reg<__half, 0>(W, N, K, smooth, q, scales, s);
+    WQ_LAUNCH_CHECK("quantize_rows_reg_kernel");
+    return WQ_OK;
+  }
   const int grid = int(N < int64_t(sm_count()) * 16 ? N : int64_t(sm_count()) * 16);
   int* st = status_ptr();
   auto* qo = static_cast<int8_t*>(q);
@@ -895,6 +1077,14 @@ int launch_quantize_rows_i8(const void* W, int w_dtype, int64_t N, int64_t K, bo
 
 int launch_quantize_rows_fp8(const void* W, int w_dtype, int64_t R, int64_t K, void* q,
                              void* scales, cudaStream_t s) {
+  if (rows_in_registers(w_dtype, K)) {
+    if (w_dtype == WQ_BF16)
+      launch_rows_reg<__nv_bfloat16, 1>(W, R, K, nullptr, q, scales, s);
+    else
+      launch_rows_reg<__half, 1>(W, R, K, nullptr, q, scales, s);
+    WQ_LAUNCH_CHECK("quantize_rows_reg_kernel");
+    return WQ_OK;
+  }
   const int grid = int(R < int64_t(sm_count()) * 16 ? R : int64_t(sm_count()) * 16);
   int* st = status_ptr();
   auto* qo = static_cast<uint8_t*>(q);

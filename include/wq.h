@@ -116,11 +116,11 @@ WQ_API int wq_dequant(const void *codes, const void *scales, const void *zeros,
  * group_size == 128 (others: WQ_ERR_UNSUPPORTED, [P4] sec. 7.2: the group must
  * divide the kernel tile); Y bf16 [M, N]; fp32 accumulation.
  * M <= 16 runs a decode kernel (every weight byte streamed once from HBM,
- * the work split evenly over all SMs) on the CUDA cores at M <= 2 (and at
- * M <= 4 when K <= 8192 and N * K <= 2^26) while the prepared X (two int8
- * limbs per element) fits in shared memory -- K <= 75776 at M = 1, 37888 at
- * M = 2, 24576 at M = 3, 18432 at M = 4 -- and on the tensor cores otherwise;
- * larger M runs the tensor-core GEMM.
+ * the work split evenly over all SMs): on the CUDA cores at M <= 4 while a
+ * CTA's fp32 row partials (ceil(N / (4 P)) * 4 rows x ceil(K / 1024) chunks x
+ * M rounded up to 1, 2 or 4, P = the SM count) fit in shared memory beside
+ * its ring (about 160 KB; N = 28672 and K = 28672 both fit with a wide
+ * margin), on the tensor cores otherwise; larger M runs the tensor-core GEMM.
  * Requires K % 128 == 0 and N % 8 == 0.
  *
  * Stream order: the CUDA-core decode kernel is launched as a programmatic
@@ -150,21 +150,25 @@ WQ_API int wq_gemm_w4a16(const void *X, int64_t M, int64_t K, const void *codes,
 
 /*
  * wq_gemm_w4a16_noalloc -- the decode product of wq_gemm_w4a16 (M = 1..16)
- * for callers that cannot allocate device memory: code running while a CUDA
- * graph is being captured (cudaMalloc is not allowed there), serving loops
- * whose device memory belongs to another allocator, C hosts without a device
- * allocator.  The quantization write-ups have no counterpart of this call.
+ * for callers that cannot hand the library any device memory: a serving loop
+ * whose device memory all belongs to another allocator under a fixed budget,
+ * a plain C host with no device allocator of its own, or a latency-critical
+ * path where a cudaMalloc (which may synchronize the device) is not
+ * acceptable.  The quantization write-ups have no counterpart of this call.
  *
  * Same arguments and results as wq_gemm_w4a16 without ws / ws_bytes.  The
  * library allocates nothing, in this call or ever: the scratch is an array of
  * 4 MiB + 4 KiB inside the library's device image, held by every GPU that
  * loads the library until the process exits.  Limits: M <= 16, N <= 131072,
- * at most 256 SMs (WQ_ERR_UNSUPPORTED beyond them).
+ * at most 256 SMs (WQ_ERR_UNSUPPORTED beyond them, before any launch).  At
+ * M <= 4 the CUDA-core kernel runs and no scratch is used.
  *
- * The first call on a device looks up the array's device address; make that
- * first call before any stream capture.  Every call shares the one array and
- * clears its counters on its own stream: calls that overlap on the GPU (other
- * streams, other host threads) race and give wrong results -- serialize them.
+ * The first call on a device does the set-up: it looks up the array's device
+ * address and sets the decode kernels' launch attributes.  Make that first
+ * call before any stream capture.  Every call shares the one array, which
+ * keeps the last call's contents; each call clears the counters that must
+ * start at zero on its own stream.  Calls that overlap on the GPU (other
+ * streams, other host threads) race and give wrong results: serialize them.
  */
 WQ_API int wq_gemm_w4a16_noalloc(const void *X, int64_t M, int64_t K,
                                  const void *codes, const void *scales,

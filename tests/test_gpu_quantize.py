@@ -272,3 +272,44 @@ def test_kv_half_way():
     np.testing.assert_array_equal(qv.cpu().numpy(), oqv)
     np.testing.assert_array_equal(sk.cpu().numpy().view(np.uint32), osk.view(np.uint32))
     np.testing.assert_array_equal(sv.cpu().numpy().view(np.uint32), osv.view(np.uint32))
+
+
+# ------------------------- per-token quantizers with the row held in registers
+# 16-bit rows of 1024, 2048, 4096 or 8192 elements go through a kernel that
+# reads each row once; its codes and scales must equal the oracle's, like the
+# two-pass kernel's (3072 and 5120 take the two-pass kernel).
+
+@pytest.mark.parametrize("M,K", [(1, 1024), (13, 2048), (7, 8192), (3, 3072), (5, 5120)])
+def test_act_quant_rows_in_registers(M, K):
+    X = make_activation(M, K, seed=M * 7 + K, outlier_dims=6)
+    X[-1, :] = 0.0   # an all-zero row takes the 1e-8 floor
+    check_act(X)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("M,K", [(5, 1024), (9, 8192)])
+def test_fp8_rows_in_registers(dtype, M, K):
+    A = make_activation(M, K, seed=M + 3 * K, outlier_dims=6, dtype=dtype)
+    q, s = wq.quantize_fp8_rows(A.cuda())
+    arr, tag = oracle_input(A)
+    oq, os_, st = oracle.quantize_fp8_rows(arr, dtype_tag=tag)
+    assert st == oracle.OK
+    np.testing.assert_array_equal(q.cpu().numpy(), oq)
+    np.testing.assert_array_equal(s.cpu().numpy(), os_)
+
+
+def test_act_quant_rows_in_registers_non_finite():
+    """An infinity counts in the row maximum and a NaN does not, as in the
+    oracle; the codes of such rows still match it and the status reports the
+    non-finite input."""
+    X = make_activation(4, 1024, seed=9).float()
+    X[1, 10] = float("inf")
+    X[2, 20] = float("nan")
+    X = X.to(torch.bfloat16)
+    wq.wq_get_device_status(reset=True)
+    q, s = wq.quant_act_i8(X.cuda())
+    assert wq.wq_get_device_status(reset=True) == wq.WQ_ERR_NONFINITE
+    oq, os_, st = oracle.quant_act_i8(bf16_bits(X), dtype_tag=oracle.BF16)
+    assert st == oracle.ERR_NONFINITE
+    np.testing.assert_array_equal(q.cpu().numpy(), oq)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
