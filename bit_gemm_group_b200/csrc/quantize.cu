@@ -182,33 +182,19 @@ __device__ __forceinline__ void unpack2<__half>(uint32_t w, float& a, float& b) 
   b = f.y;
 }
 
-// acc' = w * 0 + acc on the two 16-bit lanes: stays (+-)0 while every element
-// seen is finite and turns NaN, for good, at the first Inf or NaN.
-template <typename T>
-__device__ __forceinline__ uint32_t nonfinite_acc(uint32_t acc, uint32_t w);
-template <>
-__device__ __forceinline__ uint32_t nonfinite_acc<__nv_bfloat16>(uint32_t acc, uint32_t w) {
-  __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&acc);
-  a = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&w), __float2bfloat162_rn(0.f), a);
-  return *reinterpret_cast<const uint32_t*>(&a);
-}
-template <>
-__device__ __forceinline__ uint32_t nonfinite_acc<__half>(uint32_t acc, uint32_t w) {
-  __half2 a = *reinterpret_cast<const __half2*>(&acc);
-  a = __hfma2(*reinterpret_cast<const __half2*>(&w), __float2half2_rn(0.f), a);
-  return *reinterpret_cast<const uint32_t*>(&a);
-}
-__device__ __forceinline__ bool is_nonfinite_acc(uint32_t acc) { return (acc & 0x7FFF7FFFu) != 0; }
-
 // rint(fl(x / s)) for an INT8 code, from inv = rcp_approx(s).  Exact for
-// |x/s| <= 128.5: r = x * inv is within 2^-15.4 of x/s and fl(x/s) within
-// 2^-17, so rint(r) is the IEEE result unless r is within 2^-14 of a
-// half-integer, where the division itself decides.  Larger quotients
-// saturate the code either way.
+// |x/s| <= 128.5; larger quotients saturate the code either way.
 __device__ __forceinline__ float rint_quot_i8(float x, float s, float inv) {
-  const float r = x * inv;
-  const float k = rintf(r);
-  if (fabsf(fabsf(r - k) - 0.5f) <= 0x1p-14f) return rintf(div_rn(x, s));
+  // k = rint of the exact product x * inv (one fma with 1.5 2^23); d, the
+  // residual x * inv - k rounded once, is within 2^-24 of the true one.  The
+  // reciprocal is within one ulp, so x * inv is within 1.01 2^-16 of x / s,
+  // and fl(x / s) within 2^-17 more: when |d| is below 0.5 - 2^-14, fl(x / s)
+  // lies on k's side of the half-integers and rounds to k as well; otherwise
+  // the division decides.
+  const float magic = 12582912.f;  // 1.5 * 2^23
+  const float k = fmaf(x, inv, magic) - magic;
+  const float d = fmaf(x, inv, -k);
+  if (fabsf(d) >= 0.5f - 0x1p-14f) return rintf(div_rn(x, s));
   return k;
 }
 
@@ -236,30 +222,118 @@ __device__ __forceinline__ float quot_e4m3(float x, float s, float inv) {
 // loads, one 8-byte store of codes); a warp takes 32 / LPG adjacent groups per
 // step and U steps are loaded before any is processed.
 //
-// Exactness of the reciprocal multiply here: x is a 16-bit float and s an
-// fp16 scale, x = mx 2^a and s = ms 2^b with integer significands below 2^11.
-// Then x/s - (j + 1/2) is a multiple of 2^min(a - b, -1) / ms, so x/s is
-// either exactly a half-integer or more than 2^-14 away from every one (the
-// bound holds for every 16-bit x against every finite fp16 s; codes only
-// depend on |x/s| <= 24, beyond which the clamp saturates them either way,
-// and there r is within 2^-17.4 of x/s).  rint(r) is therefore exact except
-// at exact half-integers, which are recognised without rounding: with
-// k = rint(r), e = x - k s is exact in one fma (x and k s are within a factor
-// of two, or k = 0), and x/s is a half-integer iff |e| = s/2; the IEEE result
-// is then the even one of k and k + sign(e).
-template <typename T, int LPG, int U>
+// Codes are the IEEE quotient fl(x / s) itself, rounded to nearest even,
+// obtained without a division: with y = rcp_approx(s) (within one ulp),
+// q0 = fl(x y) is within 3 ulp of x/s, the residual r = x - q0 s is exact in
+// one fma (fewer than 3 * 2^12 units of the last place of q0 s or of x), and
+// q0 + r y is within 2^-21 ulp of x/s.  For x a 16-bit float and s an fp16
+// value (significands of at most 11 bits) x/s is never an fp32 rounding
+// midpoint and lies at least 2^-12 ulp from every one, so fl(q0 + r y) is
+// fl(x / s) exactly (Markstein's correction step).  fl(x / s) + 1.5 2^23
+// then rounds to even at unit spacing, and its bit pattern is 0x4B400000 plus
+// the integer code; codes of |x/s| below 2^-10 are 0 whatever the last bits.
+// A quotient that exact half-way tests used to settle is now exact as it
+// stands: x/s = j + 1/2 is an fp32 number and the add rounds it to even.
+__device__ __forceinline__ float quot16(float x, float s, float y) {
+  const float q0 = x * y;
+  const float r = fmaf(-q0, s, x);
+  return fmaf(r, y, q0);
+}
+
+// The largest |x| (sym) or the smallest and largest x (asym) of a lane's 16
+// 16-bit elements, on the packed pairs.  NaN propagates (.NaN), so a lane
+// with a NaN or an infinity yields a non-finite statistic.
+template <typename T>
+__device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b);
+template <>
+__device__ __forceinline__ uint32_t absmax2<__nv_bfloat16>(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+template <>
+__device__ __forceinline__ uint32_t absmax2<__half>(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+template <typename T>
+__device__ __forceinline__ uint32_t min2(uint32_t a, uint32_t b);
+template <typename T>
+__device__ __forceinline__ uint32_t max2(uint32_t a, uint32_t b);
+template <>
+__device__ __forceinline__ uint32_t min2<__nv_bfloat16>(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+template <>
+__device__ __forceinline__ uint32_t max2<__nv_bfloat16>(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+template <>
+__device__ __forceinline__ uint32_t min2<__half>(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.NaN.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+template <>
+__device__ __forceinline__ uint32_t max2<__half>(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// sum over e = 0..7 of 0x4B400000 * 16^e, modulo 2^32: what eight codes'
+// fp32 patterns add to a packed word beyond the codes themselves
+__host__ __device__ constexpr uint32_t magic_nibble_sum() {
+  uint32_t c = 0u;
+  for (int e = 0; e < 8; ++e) c += 0x4B400000u << (4 * e);
+  return c;
+}
+
+// The 16 codes of a lane as two packed words: nibble e of word h holds
+// clamp(code, lo, hi) + zq for element 8 h + e, where the pattern of
+// fl(x / s) + 1.5 2^23 (clamped to [1.5 2^23 + lo, 1.5 2^23 + hi] when
+// CLAMP) is added in at bit 4 e; the pattern's constant part is taken out
+// once per word (the sum stays exact modulo 2^32 and no nibble borrows).
+template <typename T, bool CLAMP>
+__device__ __forceinline__ uint2 pack_codes16(const uint32_t (&w)[8], float s, float y,
+                                              float tlo, float thi, int zq) {
+  constexpr float magic = 12582912.f;  // 1.5 * 2^23
+  uint32_t acc[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float a, b;
+    unpack2<T>(w[i], a, b);
+    float ta = quot16(a, s, y) + magic;
+    float tb = quot16(b, s, y) + magic;
+    if (CLAMP) {
+      ta = fminf(fmaxf(ta, tlo), thi);
+      tb = fminf(fmaxf(tb, tlo), thi);
+    }
+    acc[i >> 2] += (__float_as_uint(ta) << (8 * (i & 3))) +
+                   (__float_as_uint(tb) << (8 * (i & 3) + 4));
+  }
+  const uint32_t off = uint32_t(zq) * 0x11111111u - magic_nibble_sum();
+  return make_uint2(acc[0] + off, acc[1] + off);
+}
+
+template <typename T, bool SYM, int LPG, int U>
 __global__ void __launch_bounds__(256) quantize_int4_x16_kernel(
-    const T* __restrict__ W, int64_t total_groups, int sym, uint8_t* __restrict__ codes,
+    const T* __restrict__ W, int64_t total_groups, uint8_t* __restrict__ codes,
     __half* __restrict__ scales, __half* __restrict__ zeros, int* status) {
   constexpr int GS = 16 * LPG;   // group size
   constexpr int GPW = 32 / LPG;  // groups per warp and step
+  constexpr float magic = 12582912.f;
   const int lane = threadIdx.x & 31;
   const int sub = lane / LPG, li = lane % LPG;
   const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
-  const int qmin = sym ? -8 : 0;
-  uint32_t nf = 0;
-  bool inf_scale = false;
+  constexpr int qmin = SYM ? -8 : 0;
+  bool bad = false;
 
   for (int64_t base = warp * (U * GPW); base < total_groups; base += nwarps * (U * GPW)) {
     uint4 in[U][2];
@@ -281,20 +355,17 @@ __global__ void __launch_bounds__(256) quantize_int4_x16_kernel(
       const bool live = gi < total_groups;
       const uint32_t w[8] = {in[j][0].x, in[j][0].y, in[j][0].z, in[j][0].w,
                              in[j][1].x, in[j][1].y, in[j][1].z, in[j][1].w};
-      float x[16];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        unpack2<T>(w[i], x[2 * i], x[2 * i + 1]);
-        nf = nonfinite_acc<T>(nf, w[i]);
-      }
       unsigned short s_bits;
       float sf;
       int z = 0;
       bool degenerate;
-      if (sym) {
-        float amax = 0.f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(x[e]));
+      if (SYM) {
+        uint32_t m = absmax2<T>(absmax2<T>(absmax2<T>(w[0], w[1]), absmax2<T>(w[2], w[3])),
+                                absmax2<T>(absmax2<T>(w[4], w[5]), absmax2<T>(w[6], w[7])));
+        float ma, mb;
+        unpack2<T>(m, ma, mb);
+        float amax = fmaxf(fabsf(ma), fabsf(mb));
+        bad |= !(amax <= 3.402823466e38f);  // Inf or NaN in the lane
 #pragma unroll
         for (int o = LPG / 2; o > 0; o >>= 1)
           amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -302,12 +373,16 @@ __global__ void __launch_bounds__(256) quantize_int4_x16_kernel(
         degenerate = (amax < 1e-8f) || (sf == 0.f);
         if (degenerate) sf = f16_round_trip(amax, &s_bits);
       } else {
-        float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          mn = fminf(mn, x[e]);
-          mx = fmaxf(mx, x[e]);
-        }
+        uint32_t lo2 = min2<T>(min2<T>(min2<T>(w[0], w[1]), min2<T>(w[2], w[3])),
+                               min2<T>(min2<T>(w[4], w[5]), min2<T>(w[6], w[7])));
+        uint32_t hi2 = max2<T>(max2<T>(max2<T>(w[0], w[1]), max2<T>(w[2], w[3])),
+                               max2<T>(max2<T>(w[4], w[5]), max2<T>(w[6], w[7])));
+        float a, b, c, d;
+        unpack2<T>(lo2, a, b);
+        unpack2<T>(hi2, c, d);
+        float mn = fminf(a, b), mx = fmaxf(c, d);
+        bad |= !(fabsf(a) <= 3.402823466e38f && fabsf(b) <= 3.402823466e38f &&
+                 fabsf(c) <= 3.402823466e38f && fabsf(d) <= 3.402823466e38f);
 #pragma unroll
         for (int o = LPG / 2; o > 0; o >>= 1) {
           mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -325,38 +400,29 @@ __global__ void __launch_bounds__(256) quantize_int4_x16_kernel(
       }
       if (live && li == 0) {
         scales[gi] = __ushort_as_half(s_bits);
-        if (!sym) zeros[gi] = __int2half_rn(z);
+        if (!SYM) zeros[gi] = __int2half_rn(z);
       }
-      inf_scale |= isinf(sf);
-      const float inv = rcp_approx(sf), hs = 0.5f * sf;
-      float k[16];
-      bool tie = false;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        k[e] = rintf(x[e] * inv);
-        tie |= fabsf(fmaf(-k[e], sf, x[e])) == hs;
-      }
-      if (__any_sync(0xffffffffu, tie)) {  // exact half-way quotients: to even
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float d = fmaf(-k[e], sf, x[e]);
-          if (fabsf(d) == hs && (int(k[e]) & 1)) k[e] += copysignf(1.f, d);
-        }
-      }
+      bad |= isinf(sf);
+      // a degenerate group takes code 0 for every element (y = 0)
+      const float y = degenerate ? 0.f : rcp_approx(sf);
       const int zq = z - qmin;  // nibble = clamp(q + z, qmin, qmax) - qmin
-      uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int nib =
-            degenerate ? -qmin : min(max(__float2int_rn(fminf(k[e], 64.f)) + zq, 0), 15);
-        packed[e >> 3] |= uint32_t(nib) << (4 * (e & 7));
+      const float tlo = magic - float(zq), thi = magic + float(15 - zq);
+      uint2 packed;
+      if (SYM) {
+        // |x/s| <= amax/s < 7.5 for a normal fp16 s = fl16(amax / 7): no clamp;
+        // a subnormal s (amax below 4.3e-4) can reach +-8 and takes it
+        const bool clamp = !degenerate && sf < 0x1p-14f;
+        if (__any_sync(0xffffffffu, clamp))
+          packed = pack_codes16<T, true>(w, sf, y, tlo, thi, zq);
+        else
+          packed = pack_codes16<T, false>(w, sf, y, tlo, thi, zq);
+      } else {
+        packed = pack_codes16<T, true>(w, sf, y, tlo, thi, zq);
       }
-      if (live)
-        *reinterpret_cast<uint2*>(codes + gi * (GS / 2) + li * 8) = make_uint2(packed[0], packed[1]);
+      if (live) *reinterpret_cast<uint2*>(codes + gi * (GS / 2) + li * 8) = packed;
     }
   }
-  if (__any_sync(0xffffffffu, is_nonfinite_acc(nf) || inf_scale) && lane == 0)
-    record_error(status, WQ_ERR_NONFINITE);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(status, WQ_ERR_NONFINITE);
 }
 
 // ---------------------------------------------------------------------------
@@ -975,9 +1041,15 @@ static void quantize_int4_x16(const void* W, int64_t N, int64_t K, int sym, void
   constexpr int U = 4;
   const int64_t total = N * (K / (16 * LPG));
   const int64_t steps = (total + U * (32 / LPG) - 1) / (U * (32 / LPG));  // warp steps
-  wq::quantize_int4_x16_kernel<T, LPG, U><<<grid_for(steps, 8), 256, 0, s>>>(
-      static_cast<const T*>(W), total, sym, static_cast<uint8_t*>(codes),
-      static_cast<__half*>(scales), static_cast<__half*>(zeros), status_ptr());
+  const int grid = grid_for(steps, 8);
+  if (sym)
+    wq::quantize_int4_x16_kernel<T, true, LPG, U><<<grid, 256, 0, s>>>(
+        static_cast<const T*>(W), total, static_cast<uint8_t*>(codes),
+        static_cast<__half*>(scales), static_cast<__half*>(zeros), status_ptr());
+  else
+    wq::quantize_int4_x16_kernel<T, false, LPG, U><<<grid, 256, 0, s>>>(
+        static_cast<const T*>(W), total, static_cast<uint8_t*>(codes),
+        static_cast<__half*>(scales), static_cast<__half*>(zeros), status_ptr());
 }
 
 template <typename T>

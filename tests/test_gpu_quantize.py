@@ -199,6 +199,42 @@ def test_int4_half_way_quotients(dtype, g):
     check_int4(Wa.to(dtype), g, sym=False)
 
 
+def _scale_sweep(rows, K, g, dtype, seed):
+    """Groups over a wide range of scales (log-uniform over 2^-22 .. 2^8 of
+    the target step, fp16 subnormal scales included), half of them with a
+    step of at most 4 significant bits so that (j + 1/2) step is exact in the
+    16-bit type (exact half-way quotients), the other half with random
+    steps; the elements are j + 1/2 + d steps, d from {0, +-2^-12, +-2^-9,
+    uniform(-1/2, 1/2)}, rounded to the type, so quotients crowd around
+    rounding points.  Element 0 of each group is 7 steps (sym amax) and
+    element 1 is -8 or -7 steps (asym minimum)."""
+    rng = np.random.default_rng(seed)
+    ng = rows * K // g
+    hi_exp = 8 if dtype == torch.bfloat16 else 5
+    e = rng.uniform(-22, hi_exp, ng)
+    frac = np.where(rng.random(ng) < 0.5, np.round(rng.uniform(8, 16, ng)) / 8,
+                    rng.uniform(1, 2, ng))
+    step = (frac * np.exp2(np.floor(e))).astype(np.float32).astype(np.float64)
+    j = rng.integers(-8, 8, (ng, g)).astype(np.float64)
+    d = rng.choice([0.0, 2.0 ** -12, -2.0 ** -12, 2.0 ** -9, -2.0 ** -9, np.nan], (ng, g))
+    u = rng.uniform(-0.5, 0.5, (ng, g))
+    d = np.where(np.isnan(d), u, d)
+    v = (j + 0.5 + d) * step[:, None]
+    v[:, 0] = 7 * step
+    v[:, 1] = np.where(rng.random(ng) < 0.5, -8, -7) * step
+    return torch.from_numpy(v.reshape(rows, K).astype(np.float32)).to(dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("g", [32, 128, 512])
+def test_int4_scale_sweep(dtype, g):
+    """Codes follow the IEEE quotient across scales and near every rounding
+    point (subnormal fp16 scales take the clamped path)."""
+    W = _scale_sweep(256, 4096, g, dtype, seed=g)
+    check_int4(W, g, sym=True)
+    check_int4(W, g, sym=False)
+
+
 def _rows_with(X):
     check_int8_rows(X)
     if X.dtype != torch.bfloat16:  # the activation quantizer takes bf16 only
