@@ -19,6 +19,13 @@ int launch_smooth_scales(const float* act, const float* w, int64_t K, float alph
                          cudaStream_t s);
 int launch_quant_kv(const void* Kc, const void* Vc, int dtype, int64_t BH, int64_t S, int64_t D,
                     void* qk, void* sk, void* qv, void* sv, cudaStream_t s);
+// One-launch KV quantizer for 16-bit caches with D in {16, 32, 64, 128, 256}
+// and S <= 16384 (kv_fused_plan picks the cluster size, the tokens per CTA and
+// the channel block); WQ_ERR_UNSUPPORTED otherwise, and launch_quant_kv takes
+// the multi-kernel path instead.
+bool kv_fused_plan(int dtype, int64_t BH, int64_t S, int64_t D, int* CS, int* R, int* CW);
+int launch_quant_kv_fused(const void* Kc, const void* Vc, int dtype, int64_t BH, int64_t S,
+                          int64_t D, void* qk, void* sk, void* qv, void* sv, cudaStream_t s);
 int launch_quantize_rows_fp8(const void* W, int w_dtype, int64_t R, int64_t K, void* q,
                              void* scales, cudaStream_t s);
 size_t gptq_workspace_bytes(int64_t N, int64_t K);

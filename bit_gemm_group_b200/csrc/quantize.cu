@@ -13,6 +13,7 @@
 // see the section below).
 #include "common.cuh"
 #include "kernels.h"
+#include "qmath.cuh"
 #include <cuda_fp8.h>
 
 namespace wq {
@@ -150,71 +151,6 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Reciprocal-multiply quantization with the IEEE-division result
-// ---------------------------------------------------------------------------
-// The quantizers' codes are defined by round-half-even of the binary32
-// quotient fl(x / s).  One reciprocal per scale and one multiply per element
-// reach the same codes: r = x * rcp(s), with rcp within one ulp of 1/s, is
-// within |x/s| * 1.5 * 2^-23 of x/s, and rint(fl(x/s)) depends only on which
-// side of each half-integer x/s lies.  So rint(r) is the IEEE result unless
-// x/s is very close to (or exactly on) a half-integer; each kernel below
-// recognises those elements and decides them exactly.
-
-// 1/v within one ulp (a single instruction).
-__device__ __forceinline__ float rcp_approx(float v) {
-  float r;
-  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
-  return r;
-}
-
-// The two 16-bit floats of a 32-bit word as fp32 (element 0 = low half).
-template <typename T>
-__device__ __forceinline__ void unpack2(uint32_t w, float& a, float& b);
-template <>
-__device__ __forceinline__ void unpack2<__nv_bfloat16>(uint32_t w, float& a, float& b) {
-  a = __uint_as_float(w << 16);
-  b = __uint_as_float(w & 0xFFFF0000u);
-}
-template <>
-__device__ __forceinline__ void unpack2<__half>(uint32_t w, float& a, float& b) {
-  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
-  a = f.x;
-  b = f.y;
-}
-
-// rint(fl(x / s)) for an INT8 code, from inv = rcp_approx(s).  Exact for
-// |x/s| <= 128.5; larger quotients saturate the code either way.
-__device__ __forceinline__ float rint_quot_i8(float x, float s, float inv) {
-  // k = rint of the exact product x * inv (one fma with 1.5 2^23); d, the
-  // residual x * inv - k rounded once, is within 2^-24 of the true one.  The
-  // reciprocal is within one ulp, so x * inv is within 1.01 2^-16 of x / s,
-  // and fl(x / s) within 2^-17 more: when |d| is below 0.5 - 2^-14, fl(x / s)
-  // lies on k's side of the half-integers and rounds to k as well; otherwise
-  // the division decides.
-  const float magic = 12582912.f;  // 1.5 * 2^23
-  const float k = fmaf(x, inv, magic) - magic;
-  const float d = fmaf(x, inv, -k);
-  if (fabsf(d) >= 0.5f - 0x1p-14f) return rintf(div_rn(x, s));
-  return k;
-}
-
-// A binary32 quotient that rounds to the same E4M3 code as fl(x / s), from
-// inv = rcp_approx(s).  r = x * inv is within 3 units of the binary32 last
-// place of x/s, and fl(x/s) within half a unit; an E4M3 half-way point in the
-// normal range has the low 20 mantissa bits 0x80000 (bit 19 alone), so when
-// r's low 20 bits are more than 4 units from that pattern, r and fl(x/s) lie
-// on the same side of every half-way point and round to the same code
-// (powers of two, where the binade changes, are codes themselves).  Nonzero
-// |r| < 2^-6 (the E4M3 subnormal range, uniform spacing 2^-9) and the rare
-// near-half-way r take the division itself.
-__device__ __forceinline__ float quot_e4m3(float x, float s, float inv) {
-  const float r = x * inv;
-  const int m20 = int(__float_as_uint(r) & 0xFFFFFu) - 0x80000;
-  if ((r != 0.f && fabsf(r) < 0x1p-6f) || (m20 >= -4 && m20 <= 4)) return div_rn(x, s);
-  return r;
-}
-
-// ---------------------------------------------------------------------------
 // INT4 group-wise quantize + pack of 16-bit weights (bf16 / fp16), g <= 512
 // ---------------------------------------------------------------------------
 // Codes, scales and zeros equal quantize_int4_kernel's bit for bit.  Lane l
@@ -238,52 +174,6 @@ __device__ __forceinline__ float quot16(float x, float s, float y) {
   const float q0 = x * y;
   const float r = fmaf(-q0, s, x);
   return fmaf(r, y, q0);
-}
-
-// The largest |x| (sym) or the smallest and largest x (asym) of a lane's 16
-// 16-bit elements, on the packed pairs.  NaN propagates (.NaN), so a lane
-// with a NaN or an infinity yields a non-finite statistic.
-template <typename T>
-__device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b);
-template <>
-__device__ __forceinline__ uint32_t absmax2<__nv_bfloat16>(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-template <>
-__device__ __forceinline__ uint32_t absmax2<__half>(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("max.NaN.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-template <typename T>
-__device__ __forceinline__ uint32_t min2(uint32_t a, uint32_t b);
-template <typename T>
-__device__ __forceinline__ uint32_t max2(uint32_t a, uint32_t b);
-template <>
-__device__ __forceinline__ uint32_t min2<__nv_bfloat16>(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("min.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-template <>
-__device__ __forceinline__ uint32_t max2<__nv_bfloat16>(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-template <>
-__device__ __forceinline__ uint32_t min2<__half>(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("min.NaN.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-template <>
-__device__ __forceinline__ uint32_t max2<__half>(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("max.NaN.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
 }
 
 // sum over e = 0..7 of 0x4B400000 * 16^e, modulo 2^32: what eight codes'
@@ -712,25 +602,41 @@ __global__ void __launch_bounds__(256) quantize_rows_reg_kernel(
       scales[r] = s;
       if (bad) record_error(status, WQ_ERR_NONFINITE);
     }
-    if (live) {
+    if (live) {  // warp-uniform: a row spans whole warps
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         union {
           uint2 v2;
           uint8_t b[8];
         } o;
+        uint32_t near = 0u;
+        if (KIND == 0 && !bad) {
+          // finite row: |x / s| <= 127.5, codes through the fp32 patterns
+          uint32_t c[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (KIND == 0) {
-            float rr = rint_quot_i8(x[8 * i + e], s, inv);
-            rr = fmaxf(-200.f, fminf(200.f, rr));
-            o.b[e] = uint8_t(int8_t(min(max(int(rr), -128), 127)));
-          } else {
-            o.b[e] = uint8_t(__nv_cvt_float_to_fp8(quot_e4m3(x[8 * i + e], s, inv),
-                                                   __NV_SATFINITE, __NV_E4M3));
+          for (int e = 0; e < 8; ++e) c[e] = code_i8_fast(x[8 * i + e], inv, near, e);
+          o.v2 = make_uint2(low_bytes4(c[0], c[1], c[2], c[3]), low_bytes4(c[4], c[5], c[6], c[7]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (KIND == 0) {
+              o.b[e] = uint8_t(int8_t(code_i8_full(x[8 * i + e], s, inv)));
+            } else {
+              o.b[e] = uint8_t(__nv_cvt_float_to_fp8(quot_e4m3(x[8 * i + e], s, inv),
+                                                     __NV_SATFINITE, __NV_E4M3));
+            }
           }
         }
-        *reinterpret_cast<uint2*>(q + r * int64_t(K) + 8 * int64_t(t + tpr * i)) = o.v2;
+        uint8_t* dst = q + r * int64_t(K) + 8 * int64_t(t + tpr * i);
+        *reinterpret_cast<uint2*>(dst) = o.v2;
+        while (near != 0u) {  // near-half-way elements, rewritten exactly
+          const int e = __ffs(near) - 1;
+          near &= near - 1u;
+          float xs[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) xs[j] = x[8 * i + j];
+          dst[e] = uint8_t(code_i8_exact(pick(xs, e), s, inv) & 0xFFu);
+        }
       }
     }
     __syncthreads();  // red[] is reused by the next rows
@@ -811,11 +717,8 @@ __global__ void __launch_bounds__(256) kv_k_absmax_kernel(const T* __restrict__ 
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float x = to_f32<T>(v.u.e[e]);
-      if (isfinite(x)) {
-        m[e] = fmaxf(m[e], fabsf(x));
-      } else {
-        bad = true;
-      }
+      bad |= !isfinite(x);
+      m[e] = fmaxf(m[e], fabsf(x));  // a NaN is skipped, an infinity counts
     }
   }
 #pragma unroll
@@ -1210,6 +1113,8 @@ int launch_channel_absmax(const void* A, int a_dtype, int64_t R, int64_t K, floa
 
 int launch_quant_kv(const void* Kc, const void* Vc, int dtype, int64_t BH, int64_t S, int64_t D,
                     void* qk, void* sk, void* qv, void* sv, cudaStream_t s) {
+  const int fused = launch_quant_kv_fused(Kc, Vc, dtype, BH, S, D, qk, sk, qv, sv, s);
+  if (fused != WQ_ERR_UNSUPPORTED) return fused;
   float* skf = static_cast<float*>(sk);
   WQ_CUDA_CHECK(cudaMemsetAsync(skf, 0, size_t(BH) * size_t(D) * 4, s));
   if (BH == 0 || S == 0) return WQ_OK;
