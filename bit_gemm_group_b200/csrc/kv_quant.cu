@@ -22,13 +22,22 @@
 namespace wq {
 namespace kvq {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;               // V rows kernel
+constexpr int kKThreads = 256;              // K cluster kernel
 constexpr int kBoxRows = 256;                // TMA box height (rows of K)
 constexpr int kMaxSlabBytes = 64 * 1024;     // shared memory for one K slab
 constexpr int kMaxCluster = 8;               // portable cluster size
+constexpr int kNearQueue = 1024;            // deferred near-half-way groups per K CTA
+constexpr int kMaxBoxes = kMaxSlabBytes / (kBoxRows * 16 * 2);  // boxes of a slab, CW >= 16
 
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+// Arrive without release: only says that this CTA's reads of the others'
+// shared memory are over (their values are already in registers), so it does
+// not wait for this CTA's global stores to drain.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -65,6 +74,33 @@ __global__ void __launch_bounds__(kThreads) kv_v_rows_kernel(const T* __restrict
   const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
   const int64_t row1 = nrows;
   bool bad = false;
+  // per warp: groups of four codes with a near-half-way element, (row << 8) |
+  // group, rewritten by the whole warp once half the queue is used
+  constexpr int kQ = 128;
+  __shared__ unsigned long long vq[kThreads / 32][kQ];
+  __shared__ int vq_n[kThreads / 32];
+  const int wib = threadIdx.x >> 5;
+  if (lane == 0) vq_n[wib] = 0;
+  __syncwarp();
+  auto flush = [&]() {
+    __syncwarp();  // the queued groups' 16-byte stores and scales are visible
+    const int n = min(vq_n[wib], kQ);
+    for (int i = lane; i < n; i += 32) {
+      const int64_t r = int64_t(vq[wib][i] >> 8);
+      const int c = 4 * int(vq[wib][i] & 0xFFu);
+      const uint2 v = *reinterpret_cast<const uint2*>(V + r * D + c);
+      const float sc = sv[r], y = rcp_approx(sc);
+      float a0, b0, a1, b1;
+      unpack2<T>(v.x, a0, b0);
+      unpack2<T>(v.y, a1, b1);
+      *reinterpret_cast<char4*>(qv + r * D + c) =
+          make_char4(code_i8_exact(a0, sc, y), code_i8_exact(b0, sc, y),
+                     code_i8_exact(a1, sc, y), code_i8_exact(b1, sc, y));
+    }
+    __syncwarp();
+    if (lane == 0) vq_n[wib] = 0;
+    __syncwarp();
+  };
   for (int64_t vb = gw * (U * RPW); vb < row1; vb += nw * (U * RPW)) {
     uint4 in[U][2];
 #pragma unroll
@@ -98,18 +134,16 @@ __global__ void __launch_bounds__(kThreads) kv_v_rows_kernel(const T* __restrict
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
       float sc = fmaxf(div_rn(amax, 127.f), 1e-8f);
       float y = rcp_approx(sc);
-      uint32_t t[16];
+      uint32_t ow[4];
       uint32_t near = 0u;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float a, b;
-        unpack2<T>(w[i], a, b);
-        t[2 * i] = code_i8_fast(a, y, near, 2 * i);
-        t[2 * i + 1] = code_i8_fast(b, y, near, 2 * i + 1);
+      for (int g = 0; g < 4; ++g) {
+        float a0, b0, a1, b1;
+        unpack2<T>(w[2 * g], a0, b0);
+        unpack2<T>(w[2 * g + 1], a1, b1);
+        ow[g] = codes_i8_x4(a0, b0, a1, b1, y, y, y, y, near, g);
       }
-      uint4 o = make_uint4(low_bytes4(t[0], t[1], t[2], t[3]), low_bytes4(t[4], t[5], t[6], t[7]),
-                           low_bytes4(t[8], t[9], t[10], t[11]),
-                           low_bytes4(t[12], t[13], t[14], t[15]));
+      uint4 o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
       if (__any_sync(0xffffffffu, special)) {
         // the row maximum by the definition (NaN skipped, infinities kept)
         const uint32_t p2 =
@@ -142,16 +176,28 @@ __global__ void __launch_bounds__(kThreads) kv_v_rows_kernel(const T* __restrict
         int8_t* dst = qv + r * D + seg * 16;
         *reinterpret_cast<uint4*>(dst) = o;
         if (seg == 0) sv[r] = sc;
-        while (near != 0u) {  // near-half-way elements, rewritten exactly
-          const int e = __ffs(near) - 1;
+        while (near != 0u) {  // groups with a near-half-way element: queued
+          const int g = __ffs(near) - 1;
           near &= near - 1u;
-          float a, b;
-          unpack2<T>(pick(w, e >> 1), a, b);
-          dst[e] = int8_t(code_i8_exact((e & 1) ? b : a, sc, y) & 0xFFu);
+          const int slot = atomicAdd(&vq_n[wib], 1);
+          if (slot < kQ) {
+            vq[wib][slot] = (static_cast<unsigned long long>(r) << 8) | unsigned(seg * 4 + g);
+            continue;
+          }
+          // queue full: rewritten here
+          float a0, b0, a1, b1;
+          unpack2<T>(pick(w, 2 * g), a0, b0);
+          unpack2<T>(pick(w, 2 * g + 1), a1, b1);
+          *reinterpret_cast<char4*>(dst + 4 * g) =
+              make_char4(code_i8_exact(a0, sc, y), code_i8_exact(b0, sc, y),
+                         code_i8_exact(a1, sc, y), code_i8_exact(b1, sc, y));
         }
       }
     }
+    __syncwarp();
+    if (vq_n[wib] >= kQ / 2) flush();  // warp-uniform
   }
+  flush();
   if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(status, WQ_ERR_NONFINITE);
 }
 
@@ -159,19 +205,25 @@ __global__ void __launch_bounds__(kThreads) kv_v_rows_kernel(const T* __restrict
 // cluster is one head and one block of CW channels; CTA `rank` owns tokens
 // [rank R, rank R + R).
 template <typename T, int CW, int D>
-__global__ void __launch_bounds__(kThreads, 3) kv_k_cluster_kernel(
+__global__ void __launch_bounds__(kKThreads, 3) kv_k_cluster_kernel(
     const __grid_constant__ CUtensorMap kmap, int64_t S, int R, int8_t* __restrict__ qk,
     float* __restrict__ sk, int* status, uint64_t wait_ns) {
   constexpr int WPR = CW / 2;          // 32-bit words (channel pairs) per slab row
   constexpr int TPR = CW / 8;          // threads per slab row, 16 bytes each
-  constexpr int RPS = kThreads / TPR;  // slab rows per CTA step
+  constexpr int RPS = kKThreads / TPR;  // slab rows per CTA step
   extern __shared__ __align__(128) unsigned char smem_raw[];
   T* slab = reinterpret_cast<T*>(smem_raw);  // [boxes * kBoxRows][CW]
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t bars[kMaxBoxes];  // one per TMA box
   __shared__ uint32_t part[2][WPR];          // this CTA's channel-pair maxima
-  __shared__ uint32_t wred[kThreads / 32][WPR];
+  __shared__ uint32_t comb[kMaxCluster][WPR];  // the cluster's partial maxima
+  __shared__ int s_fail;
+  __shared__ uint32_t wred[kKThreads / 32][WPR];
   __shared__ float s_sc[CW], s_y[CW];
   __shared__ int s_special;
+  // groups of four codes with a near-half-way element: (slab row << 8) |
+  // first channel; rewritten by the whole CTA after the slab is quantized
+  __shared__ uint32_t nq[kNearQueue];
+  __shared__ int nq_n;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_rank();
@@ -183,38 +235,37 @@ __global__ void __launch_bounds__(kThreads, 3) kv_k_cluster_kernel(
   const int boxes = (rows + kBoxRows - 1) / kBoxRows;
 
   if (tid == 0) {
-    tc::mbar_init(&bar, 1);
+    for (int b = 0; b < boxes; ++b) tc::mbar_init(&bars[b], 1);
     tc::fence_mbar_init();
     s_special = 0;
+    s_fail = 0;
+    nq_n = 0;
   }
   __syncthreads();
   if (tid == 0) {
     tc::tma_prefetch_desc(&kmap);
-    tc::mbar_arrive_expect_tx(&bar, uint32_t(boxes) * kBoxRows * CW * sizeof(T));
-    for (int b = 0; b < boxes; ++b)
-      tc::tma_load_2d(slab + size_t(b) * kBoxRows * CW, &kmap, &bar, cb * CW,
+    for (int b = 0; b < boxes; ++b) {
+      tc::mbar_arrive_expect_tx(&bars[b], uint32_t(kBoxRows * CW * sizeof(T)));
+      tc::tma_load_2d(slab + size_t(b) * kBoxRows * CW, &kmap, &bars[b], cb * CW,
                       int32_t(bh * S + r0 + int64_t(b) * kBoxRows));
-  }
-
-  // the slab has landed: one warp waits (bounded), the block barrier releases
-  // the rest; on timeout the slab is not read
-  __shared__ int s_ok;
-  if (warp == 0) {
-    bool ok0 = true;
-    if (boxes > 0) ok0 = tc::wait_until(&bar, 0, tc::globaltimer_ns() + wait_ns);
-    if (lane == 0) {
-      s_ok = ok0 ? 1 : 0;
-      if (!ok0) record_error(status, WQ_ERR_TIMEOUT);
     }
   }
-  __syncthreads();
-  const bool ok = s_ok != 0;
 
-  // channel-pair maxima of the slab (NaN-propagating)
+  // channel-pair maxima of the slab (NaN-propagating), box by box as each
+  // lands (bounded waits; after a timeout the rest of the slab is not read)
   const int cg = tid % TPR, rl = tid / TPR;
   uint32_t m[4] = {0u, 0u, 0u, 0u};
-  if (ok) {
-    for (int r = rl; r < rows; r += RPS) {
+  const uint64_t deadline = tc::globaltimer_ns() + wait_ns;
+  for (int b = 0; b < boxes; ++b) {
+    if (!__all_sync(0xffffffffu, tc::wait_until(&bars[b], 0, deadline))) {
+      if (lane == 0) {
+        s_fail = 1;
+        record_error(status, WQ_ERR_TIMEOUT);
+      }
+      break;
+    }
+    const int rend = rows < (b + 1) * kBoxRows ? rows : (b + 1) * kBoxRows;
+    for (int r = b * kBoxRows + rl; r < rend; r += RPS) {
       const uint4 v = *reinterpret_cast<const uint4*>(slab + size_t(r) * CW + cg * 8);
       m[0] = absmax2<T>(m[0], v.x);
       m[1] = absmax2<T>(m[1], v.y);
@@ -230,18 +281,22 @@ __global__ void __launch_bounds__(kThreads, 3) kv_k_cluster_kernel(
 #pragma unroll
     for (int i = 0; i < 4; ++i) wred[warp][cg * 4 + i] = m[i];
   __syncthreads();
+  const bool ok = s_fail == 0;
   if (tid < WPR) {
     uint32_t v = wred[0][tid];
 #pragma unroll
-    for (int w = 1; w < kThreads / 32; ++w) v = absmax2<T>(v, wred[w][tid]);
+    for (int w = 1; w < kKThreads / 32; ++w) v = absmax2<T>(v, wred[w][tid]);
     part[0][tid] = v;
   }
   cluster_arrive();
   cluster_wait();  // every CTA's partial maxima are visible
 
+  // one remote load per thread, then the reduction over the ranks
+  if (tid < WPR * CS) comb[tid / WPR][tid % WPR] = ld_cluster_u32(&part[0][tid % WPR], tid / WPR);
+  __syncthreads();
   uint32_t pair = 0u;
   if (tid < WPR) {
-    for (int k = 0; k < CS; ++k) pair = absmax2<T>(pair, ld_cluster_u32(&part[0][tid], k));
+    for (int k = 0; k < CS; ++k) pair = absmax2<T>(pair, comb[k][tid]);
     float a, b;
     unpack2<T>(pair, a, b);
     if (!(fabsf(a) <= 3.402823466e38f && fabsf(b) <= 3.402823466e38f)) s_special = 1;
@@ -275,15 +330,17 @@ __global__ void __launch_bounds__(kThreads, 3) kv_k_cluster_kernel(
     if (tid < WPR) {
       uint32_t v = wred[0][tid];
 #pragma unroll
-      for (int w = 1; w < kThreads / 32; ++w) v = absmax2_skipnan<T>(v, wred[w][tid]);
+      for (int w = 1; w < kKThreads / 32; ++w) v = absmax2_skipnan<T>(v, wred[w][tid]);
       part[1][tid] = v;
     }
     cluster_arrive();
     cluster_wait();
+    if (tid < WPR * CS)
+      comb[tid / WPR][tid % WPR] = ld_cluster_u32(&part[1][tid % WPR], tid / WPR);
+    __syncthreads();
     if (tid < WPR) {
       pair = 0u;
-      for (int k = 0; k < CS; ++k)
-        pair = absmax2_skipnan<T>(pair, ld_cluster_u32(&part[1][tid], k));
+      for (int k = 0; k < CS; ++k) pair = absmax2_skipnan<T>(pair, comb[k][tid]);
     }
     if (tid == 0 && rank == 0) record_error(status, WQ_ERR_NONFINITE);
   }
@@ -301,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 3) kv_k_cluster_kernel(
       sk[bh * D + cb * CW + 2 * tid + 1] = sb;
     }
   }
-  cluster_arrive();  // this CTA is done reading the others' shared memory
+  cluster_arrive_relaxed();  // this CTA is done reading the others' shared memory
   __syncthreads();
 
   // quantize the slab: 8 channels per thread, fixed over the rows
@@ -312,51 +369,99 @@ __global__ void __launch_bounds__(kThreads, 3) kv_k_cluster_kernel(
     y[e] = s_y[cg * 8 + e];
   }
   int8_t* qk_head = qk + bh * S * D + cb * CW + cg * 8;
-  if (ok) {
-    for (int base = 0; base < rows; base += RPS) {  // warp-uniform trip count
-      const int r = base + rl;
-      const bool live = r < rows;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (live) v = *reinterpret_cast<const uint4*>(slab + size_t(r) * CW + cg * 8);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      uint2 o;
-      uint32_t near = 0u;
-      if (!special) {
-        uint32_t t[8];
+  // one slab row segment (8 channels) of this thread: codes, store, and the
+  // near-half-way groups queued
+  auto quant_row = [&](const uint4 v, const int r, const bool live) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint2 o;
+    uint32_t near = 0u;
+    if (!special) {
+      uint32_t ow[2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float a, b;
-          unpack2<T>(w[i], a, b);
-          t[2 * i] = code_i8_fast(a, y[2 * i], near, 2 * i);
-          t[2 * i + 1] = code_i8_fast(b, y[2 * i + 1], near, 2 * i + 1);
-        }
-        o = make_uint2(low_bytes4(t[0], t[1], t[2], t[3]), low_bytes4(t[4], t[5], t[6], t[7]));
-      } else {
-        uint32_t c[2] = {0u, 0u};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float a, b;
-          unpack2<T>(w[i], a, b);
-          const uint32_t ca = uint32_t(code_i8_full(a, sc[2 * i], y[2 * i])) & 0xFFu;
-          const uint32_t cb2 = uint32_t(code_i8_full(b, sc[2 * i + 1], y[2 * i + 1])) & 0xFFu;
-          c[i >> 1] |= (ca | (cb2 << 8)) << (16 * (i & 1));
-        }
-        o = make_uint2(c[0], c[1]);
+      for (int g = 0; g < 2; ++g) {
+        float a0, b0, a1, b1;
+        unpack2<T>(w[2 * g], a0, b0);
+        unpack2<T>(w[2 * g + 1], a1, b1);
+        ow[g] = codes_i8_x4(a0, b0, a1, b1, y[4 * g], y[4 * g + 1], y[4 * g + 2], y[4 * g + 3],
+                            near, g);
       }
-      if (live) {
-        int8_t* dst = qk_head + (r0 + r) * D;
-        *reinterpret_cast<uint2*>(dst) = o;
-        while (near != 0u) {  // near-half-way elements, rewritten exactly
-          const int e = __ffs(near) - 1;
-          near &= near - 1u;
-          float a, b;
-          unpack2<T>(pick(w, e >> 1), a, b);
-          dst[e] = int8_t(code_i8_exact((e & 1) ? b : a, pick(sc, e), pick(y, e)) & 0xFFu);
+      o = make_uint2(ow[0], ow[1]);
+    } else {
+      uint32_t c[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float a, b;
+        unpack2<T>(w[i], a, b);
+        const uint32_t ca = uint32_t(code_i8_full(a, sc[2 * i], y[2 * i])) & 0xFFu;
+        const uint32_t cb2 = uint32_t(code_i8_full(b, sc[2 * i + 1], y[2 * i + 1])) & 0xFFu;
+        c[i >> 1] |= (ca | (cb2 << 8)) << (16 * (i & 1));
+      }
+      o = make_uint2(c[0], c[1]);
+    }
+    int8_t* dst = qk_head + (r0 + r) * D;
+    if (live) *reinterpret_cast<uint2*>(dst) = o;
+    // groups with a near-half-way element: queued, one shared atomic per warp
+    const uint32_t bal0 = __ballot_sync(0xffffffffu, near & 1u);
+    const uint32_t bal1 = __ballot_sync(0xffffffffu, near & 2u);
+    if ((bal0 | bal1) != 0u) {
+      const uint32_t lt = (1u << lane) - 1u;
+      int base = 0;
+      if (lane == 0) base = atomicAdd(&nq_n, __popc(bal0) + __popc(bal1));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const int slot[2] = {base + __popc(bal0 & lt), base + __popc(bal0) + __popc(bal1 & lt)};
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        if (!((near >> g) & 1u)) continue;
+        if (slot[g] < kNearQueue) {
+          nq[slot[g]] = (uint32_t(r) << 8) | uint32_t(cg * 8 + 4 * g);
+          continue;
         }
+        // queue full: rewritten here
+        float a0, b0, a1, b1;
+        unpack2<T>(g ? w[2] : w[0], a0, b0);
+        unpack2<T>(g ? w[3] : w[1], a1, b1);
+        float sg[4], yg[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          sg[j] = g ? sc[4 + j] : sc[j];
+          yg[j] = g ? y[4 + j] : y[j];
+        }
+        *reinterpret_cast<char4*>(dst + 4 * g) =
+            make_char4(code_i8_exact(a0, sg[0], yg[0]), code_i8_exact(b0, sg[1], yg[1]),
+                       code_i8_exact(a1, sg[2], yg[2]), code_i8_exact(b1, sg[3], yg[3]));
       }
     }
+  };
+  if (ok) {
+    // two rows per thread and step, both loaded before either is processed
+    for (int base = 0; base < rows; base += 2 * RPS) {
+      const int ra = base + rl, rb = base + RPS + rl;
+      const bool la = ra < rows, lb = rb < rows;
+      uint4 va = make_uint4(0u, 0u, 0u, 0u), vb = va;
+      if (la) va = *reinterpret_cast<const uint4*>(slab + size_t(ra) * CW + cg * 8);
+      if (lb) vb = *reinterpret_cast<const uint4*>(slab + size_t(rb) * CW + cg * 8);
+      quant_row(va, ra, la);
+      quant_row(vb, rb, lb);
+    }
   }
-  if (!ok) tc::wait_until(&bar, 0, tc::globaltimer_ns() + tc::kDrainNs);  // own copies
+  // The queued groups, one per thread: exact codes from the slab (the group's
+  // 8-byte store above is ordered before this one by the block barrier).
+  __syncthreads();
+  const int nn = nq_n < kNearQueue ? nq_n : kNearQueue;
+  for (int i = tid; i < nn; i += kKThreads) {
+    const int r = int(nq[i] >> 8), c = int(nq[i] & 0xFFu);
+    const uint2 v = *reinterpret_cast<const uint2*>(slab + size_t(r) * CW + c);
+    float a0, b0, a1, b1;
+    unpack2<T>(v.x, a0, b0);
+    unpack2<T>(v.y, a1, b1);
+    *reinterpret_cast<char4*>(qk + bh * S * D + (r0 + r) * D + cb * CW + c) =
+        make_char4(code_i8_exact(a0, s_sc[c], s_y[c]), code_i8_exact(b0, s_sc[c + 1], s_y[c + 1]),
+                   code_i8_exact(a1, s_sc[c + 2], s_y[c + 2]),
+                   code_i8_exact(b1, s_sc[c + 3], s_y[c + 3]));
+  }
+  if (!ok)  // own copies still in flight
+    for (int b = 0; b < boxes; ++b)
+      tc::wait_until(&bars[b], 0, tc::globaltimer_ns() + tc::kDrainNs);
   cluster_wait();  // no CTA leaves while another may still read its partials
 }
 
@@ -392,7 +497,7 @@ int launch_k_cluster(const void* Kc, int64_t BH, int64_t S, int CS, int R, void*
   const int boxes = (R + wq::kvq::kBoxRows - 1) / wq::kvq::kBoxRows;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(CS), unsigned(D / CW), unsigned(BH));
-  cfg.blockDim = dim3(wq::kvq::kThreads, 1, 1);
+  cfg.blockDim = dim3(wq::kvq::kKThreads, 1, 1);
   cfg.dynamicSmemBytes = size_t(boxes) * wq::kvq::kBoxRows * CW * 2;
   cfg.stream = s;
   cudaLaunchAttribute at[1];

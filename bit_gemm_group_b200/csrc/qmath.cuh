@@ -169,27 +169,40 @@ __device__ __forceinline__ uint32_t code_i8_fix(float x, float s, float t, float
   return __float_as_uint(kk + magic);
 }
 
-// The pattern of rint(x y) + 1.5 2^23 (its low byte the INT8 code of a finite
-// x over a finite s with |x / s| <= 127.5) for element `e` of a lane's run,
-// with bit e of `near` raised when the element lies near half-way and needs
-// code_i8_exact instead.  Such elements are a few per thousand on real data
-// (x = +-amax/2 puts x / s within 2^-18 of 63.5), so the caller stores the
-// fast codes and then rewrites the flagged bytes one by one.
-__device__ __forceinline__ uint32_t code_i8_fast(float x, float y, uint32_t& near, int e) {
-  const float magic = 12582912.f;
-  const float t = fmaf(x, y, magic);
-  const float d = fmaf(x, y, magic - t);
-  if (fabsf(d) >= 0.5f - 0x1p-14f) near |= 1u << e;
-  return __float_as_uint(t);
+// Low bytes of four words, in order, as one word.
+__device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-// rint(fl(x / s)) + 1.5 2^23 as a pattern, for an element code_i8_fast
-// flagged.
-__device__ __forceinline__ uint32_t code_i8_exact(float x, float s, float y) {
+// INT8 codes of four elements (finite x over finite s, |x / s| <= 127.5) as
+// one word, from the fp32 patterns of rint(x y) + 1.5 2^23 (y = rcp_approx(s));
+// bit g of `near` is raised when one of the four lies near half-way and the
+// group needs code_i8_exact.  Near-half-way elements are a few per thousand
+// on real data (x = +-amax/2 puts x / s within 2^-18 of 63.5), so the caller
+// stores the fast codes and then rewrites the flagged groups.
+__device__ __forceinline__ uint32_t codes_i8_x4(float x0, float x1, float x2, float x3, float y0,
+                                                float y1, float y2, float y3, uint32_t& near,
+                                                int g) {
+  const float magic = 12582912.f;
+  const float t0 = fmaf(x0, y0, magic), t1 = fmaf(x1, y1, magic);
+  const float t2 = fmaf(x2, y2, magic), t3 = fmaf(x3, y3, magic);
+  const float d0 = fmaf(x0, y0, magic - t0), d1 = fmaf(x1, y1, magic - t1);
+  const float d2 = fmaf(x2, y2, magic - t2), d3 = fmaf(x3, y3, magic - t3);
+  const float m = fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fmaxf(fabsf(d2), fabsf(d3)));
+  if (m >= 0.5f - 0x1p-14f) near |= 1u << g;
+  return low_bytes4(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
+                    __float_as_uint(t3));
+}
+
+// The INT8 code rint(fl(x / s)) of one element (finite x and s, |x / s| <=
+// 127.5), from y = rcp_approx(s): the fast code unless the element is near
+// half-way, then code_i8_fix.
+__device__ __forceinline__ int8_t code_i8_exact(float x, float s, float y) {
   const float magic = 12582912.f;
   const float t = fmaf(x, y, magic);
   const float d = fmaf(x, y, magic - t);
-  return code_i8_fix(x, s, t, d);
+  const uint32_t bits = fabsf(d) >= 0.5f - 0x1p-14f ? code_i8_fix(x, s, t, d) : __float_as_uint(t);
+  return int8_t(bits & 0xFFu);
 }
 
 // a[i] for a run-time i without dynamic register indexing (rare paths only).
@@ -199,11 +212,6 @@ __device__ __forceinline__ V pick(const V (&a)[N], int i) {
 #pragma unroll
   for (int j = 1; j < N; ++j) v = (i == j) ? a[j] : v;
   return v;
-}
-
-// Low bytes of four words, in order, as one word.
-__device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
 // The INT8 code of the per-row / per-channel quantizers with every case of

@@ -517,7 +517,7 @@ __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
 }
 
 template <typename T, int KIND>
-__global__ void __launch_bounds__(256) quantize_rows_reg_kernel(
+__global__ void __launch_bounds__(256, 3) quantize_rows_reg_kernel(
     const T* __restrict__ X, int64_t rows, int K, const float* __restrict__ smooth,
     uint8_t* __restrict__ q, float* __restrict__ scales, int* status) {
   __shared__ float red[8];
@@ -612,10 +612,10 @@ __global__ void __launch_bounds__(256) quantize_rows_reg_kernel(
         uint32_t near = 0u;
         if (KIND == 0 && !bad) {
           // finite row: |x / s| <= 127.5, codes through the fp32 patterns
-          uint32_t c[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) c[e] = code_i8_fast(x[8 * i + e], inv, near, e);
-          o.v2 = make_uint2(low_bytes4(c[0], c[1], c[2], c[3]), low_bytes4(c[4], c[5], c[6], c[7]));
+          const float* xi = x + 8 * i;
+          o.v2 = make_uint2(
+              codes_i8_x4(xi[0], xi[1], xi[2], xi[3], inv, inv, inv, inv, near, 0),
+              codes_i8_x4(xi[4], xi[5], xi[6], xi[7], inv, inv, inv, inv, near, 1));
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -629,13 +629,15 @@ __global__ void __launch_bounds__(256) quantize_rows_reg_kernel(
         }
         uint8_t* dst = q + r * int64_t(K) + 8 * int64_t(t + tpr * i);
         *reinterpret_cast<uint2*>(dst) = o.v2;
-        while (near != 0u) {  // near-half-way elements, rewritten exactly
-          const int e = __ffs(near) - 1;
+        while (near != 0u) {  // groups with a near-half-way element, rewritten exactly
+          const int g = __ffs(near) - 1;
           near &= near - 1u;
-          float xs[8];
+          float xg[4];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) xs[j] = x[8 * i + j];
-          dst[e] = uint8_t(code_i8_exact(pick(xs, e), s, inv) & 0xFFu);
+          for (int j = 0; j < 4; ++j) xg[j] = g ? x[8 * i + 4 + j] : x[8 * i + j];
+          *reinterpret_cast<char4*>(dst + 4 * g) =
+              make_char4(code_i8_exact(xg[0], s, inv), code_i8_exact(xg[1], s, inv),
+                         code_i8_exact(xg[2], s, inv), code_i8_exact(xg[3], s, inv));
         }
       }
     }
