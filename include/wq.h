@@ -269,7 +269,12 @@ WQ_API int wq_gemm_w8a8_smooth(const void *X, int64_t M, int64_t K, const void *
  *                  S tokens of that head, qk = clamp(round(K / sk), -128, 127)
  * qk, qv int8 [BH, S, D]; sk fp32 [BH, D]; sv fp32 [BH, S].  Rounding is half
  * to even after one IEEE fp32 division.  Requires D % 8 == 0, D <= 256,
- * BH <= 65535.  K is read twice (its channel maxima span all S tokens).
+ * BH <= 65535.  16-bit caches with D in {16, 32, 64, 128, 256} and S <= 16384
+ * read K once (a thread-block cluster per head and channel block holds the
+ * head's K in shared memory while its channel maxima are combined); other
+ * shapes and fp32 caches read K twice (maxima, then codes).  A NaN is skipped
+ * by a maximum and an infinity counts; their codes follow the definition
+ * (a NaN quotient gives 127) and the status reports WQ_ERR_NONFINITE.
  * Keeping the most recent tokens unquantized (the page's residual window) is
  * the caller's choice of S.
  */
