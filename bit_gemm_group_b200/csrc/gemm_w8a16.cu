@@ -26,6 +26,8 @@
 //    epilogue warpgroup (fp32 accumulator x row scale -> bf16 Y).
 #include <stdlib.h>
 
+#include <algorithm>
+
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -141,6 +143,165 @@ __global__ void __launch_bounds__(256) gemv_w8a16_kernel(const __nv_bfloat16* __
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
       if (lane == 0 && m < M) Y[size_t(m) * N + n] = __float2bfloat16_rn(s * t);
+    }
+  }
+}
+
+// ------------------------------------------------ int8 decode on DP2A
+// int8 codes times X in 16-bit fixed point: for each activation row and
+// 128-element group of K, x' = rint(x 2^e) with e chosen so that the group's
+// largest |x| maps into [2^12, 2^13).  bf16 values down to 2^-5 of that
+// maximum are exact integers then; smaller ones move by at most 2^-13 of it.
+// A lane's 16 codes times x' is an exact integer below 2^24 (eight DP2A),
+// scaled by 2^-e into an fp32 accumulator.  A warp owns RB weight rows and
+// walks K in 512-wide chunks (16 codes per lane and row, one 16-byte load),
+// converting X once per chunk for all RB rows; the next chunk's codes are
+// loaded before the current one is multiplied.  A chunk whose X holds a NaN
+// or an infinity is multiplied in fp32 instead (the exact-code expansion).
+__device__ __forceinline__ int dp2a_lo_ss(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.lo.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp2a_hi_ss(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.hi.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// One activation row's chunk of X for this lane (16 elements at k0), in
+// fixed point: xq[j] holds x'(2j) | x'(2j + 1) << 16, inv = 2^-e.  Returns
+// false (warp-uniformly) when the chunk holds a non-finite value.
+__device__ __forceinline__ bool x_fixed_chunk(const uint4 xa, const uint4 xb, uint32_t (&xq)[8],
+                                              float& inv, float (&xf)[16]) {
+  const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+  uint32_t m2 = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(xw[0], xw[1]), bf16x2_absmax(xw[2], xw[3])),
+                              bf16x2_absmax(bf16x2_absmax(xw[4], xw[5]), bf16x2_absmax(xw[6], xw[7])));
+  float amax = fmaxf(fabsf(__uint_as_float(m2 << 16)), fabsf(__uint_as_float(m2 & 0xFFFF0000u)));
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    xf[2 * j] = __uint_as_float(xw[j] << 16);
+    xf[2 * j + 1] = __uint_as_float(xw[j] & 0xFFFF0000u);
+  }
+  bool finite = true;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) finite &= fabsf(xf[e]) <= 3.402823466e38f;
+  if (!__all_sync(0xffffffffu, finite)) return false;
+  // e = 12 - floor(log2 amax) (amax >= 2^-133 for a nonzero bf16); 2^e is
+  // applied as two exact power-of-two factors, 2^-e built from its bits
+  const int E = amax > 0.f ? int((__float_as_uint(amax) >> 23) & 0xFFu) - 127 : 0;
+  const int ee = amax > 0.f ? (E < -126 ? 130 + __clz(int(__float_as_uint(amax) & 0x7FFFFFu)) : 12 - E) : 0;
+  const int e1 = ee / 2, e2 = ee - e1;
+  const float s1 = __uint_as_float(uint32_t(127 + e1) << 23);
+  const float s2 = __uint_as_float(uint32_t(127 + e2) << 23);
+  inv = ee <= 126 ? __uint_as_float(uint32_t(127 - ee) << 23) : __uint_as_float(1u << (149 - ee));
+  const float magic = 12582912.f;  // 1.5 * 2^23
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float ta = fmaf(xf[2 * j] * s1, s2, magic);
+    const float tb = fmaf(xf[2 * j + 1] * s1, s2, magic);
+    xq[j] = prmt(__float_as_uint(ta), __float_as_uint(tb), 0x5410u);
+  }
+  return true;
+}
+
+template <int MT, int RB>
+__global__ void __launch_bounds__(256, 2) gemv_w8a16_dp_kernel(const __nv_bfloat16* __restrict__ X,
+                                                               int M, int K,
+                                                               const uint8_t* __restrict__ Wq,
+                                                               const float* __restrict__ sw, int N,
+                                                               __nv_bfloat16* __restrict__ Y) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  const int nchunk = (K + 511) / 512;
+  const int64_t nblocks = (int64_t(N) + RB - 1) / RB;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (gw >= nblocks) asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int64_t rb = gw; rb < nblocks; rb += nw) {  // warp-uniform
+    const int64_t r0 = rb * RB;
+    float acc[RB][MT];
+#pragma unroll
+    for (int r = 0; r < RB; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
+    auto load = [&](uint4 (&dst)[RB], int c) {
+      const int k0 = c * 512 + lane * 16;
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        const int64_t n = r0 + r;
+        dst[r] = (k0 < K && n < N)
+                     ? __ldcs(reinterpret_cast<const uint4*>(Wq + n * int64_t(K) + k0))
+                     : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    auto multiply = [&](const uint4 (&cw)[RB], int c) {
+      const int k0 = c * 512 + lane * 16;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        if (m >= M) break;  // uniform
+        uint4 xa = make_uint4(0u, 0u, 0u, 0u), xb = xa;
+        if (k0 < K) {
+          const uint4* xp = reinterpret_cast<const uint4*>(X + size_t(m) * K + k0);
+          xa = __ldg(xp);
+          xb = __ldg(xp + 1);
+        }
+        uint32_t xq[8];
+        float inv, xf[16];
+        if (x_fixed_chunk(xa, xb, xq, inv, xf)) {
+#pragma unroll
+          for (int r = 0; r < RB; ++r) {
+            const uint32_t w4[4] = {cw[r].x, cw[r].y, cw[r].z, cw[r].w};
+            int isum = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              isum = dp2a_lo_ss(xq[2 * j], w4[j], isum);
+              isum = dp2a_hi_ss(xq[2 * j + 1], w4[j], isum);
+            }
+            acc[r][m] = fmaf(float(isum), inv, acc[r][m]);
+          }
+        } else {  // non-finite X in this chunk: fp32 products of the exact codes
+#pragma unroll
+          for (int r = 0; r < RB; ++r) {
+            const uint32_t w4[4] = {cw[r].x, cw[r].y, cw[r].z, cw[r].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float f[4];
+              i8x4_to_f32(w4[j], f);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[r][m] = fmaf(xf[4 * j + e], f[e], acc[r][m]);
+            }
+          }
+        }
+      }
+    };
+    uint4 ca[RB], cb[RB];
+    load(ca, 0);
+    if (rb == gw) asm volatile("griddepcontrol.wait;" ::: "memory");  // X, Y after this
+    for (int c = 0; c < nchunk; c += 2) {  // ca holds chunk c, cb chunk c + 1
+      if (c + 1 < nchunk) load(cb, c + 1);
+      multiply(ca, c);
+      if (c + 1 >= nchunk) break;
+      if (c + 2 < nchunk) load(ca, c + 2);
+      multiply(cb, c + 1);
+    }
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+      const int64_t n = r0 + r;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        float t = acc[r][m];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (lane == 0 && m < M && n < N) Y[size_t(m) * N + n] = __float2bfloat16_rn(sw[n] * t);
+      }
     }
   }
 }
@@ -414,6 +575,30 @@ static int launch_w8a16_cc(const void* X, int64_t M, int64_t K, const void* Wq, 
   const auto* x = static_cast<const __nv_bfloat16*>(X);
   const auto* w = static_cast<const uint8_t*>(Wq);
   auto* y = static_cast<__nv_bfloat16*>(Y);
+  if constexpr (FMT == WQ_W8_INT8) {
+    // int8 codes: DP2A against X in fixed point, a warp per block of rows
+    const int rb = M <= 2 ? 8 : 4;
+    const int64_t warps = (N + rb - 1) / rb;
+    const int64_t cap2 = int64_t(sm_count()) * 2;
+    const int g = int(std::min<int64_t>((warps + 7) / 8, cap2));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(g), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    const int mm = int(M), kk = int(K), nn = int(N);
+    if (M == 1)
+      WQ_CUDA_CHECK(cudaLaunchKernelEx(&cfg, gemv_w8a16_dp_kernel<1, 8>, x, mm, kk, w, sw, nn, y));
+    else if (M == 2)
+      WQ_CUDA_CHECK(cudaLaunchKernelEx(&cfg, gemv_w8a16_dp_kernel<2, 8>, x, mm, kk, w, sw, nn, y));
+    else
+      WQ_CUDA_CHECK(cudaLaunchKernelEx(&cfg, gemv_w8a16_dp_kernel<4, 4>, x, mm, kk, w, sw, nn, y));
+    return WQ_OK;
+  }
   if (M == 1)
     gemv_w8a16_kernel<FMT, 1><<<grid, 256, 0, s>>>(x, int(M), int(K), w, sw, int(N), y);
   else if (M == 2)

@@ -307,8 +307,13 @@ WQ_API int wq_quantize_fp8_rows(const void *A, int a_dtype, int64_t R, int64_t K
  * them); w_scales fp32 [N]; Y bf16 [M, N].  Every code value is exact in
  * bf16, so the expanded weight is not rounded.  M <= 4 runs on the CUDA
  * cores (every weight byte streamed once), larger M on the tensor cores
- * (tcgen05.mma kind::f16).  Requires K % 64 == 0; all pointers 16-byte
- * aligned.
+ * (tcgen05.mma kind::f16).  With int8 codes and M <= 4 the CUDA-core product
+ * takes X in 16-bit fixed point, as the W4A16 decode does: per activation
+ * row and 128-element group of K, x' = rint(x 2^e) with the group's largest
+ * |x| scaled into [2^12, 2^13), exact integer dot products with the codes,
+ * scaled by 2^-e in fp32 (values below 2^-5 of the group maximum move by at
+ * most 2^-13 of it; a chunk of X holding a NaN or an infinity is multiplied
+ * in fp32).  Requires K % 64 == 0; all pointers 16-byte aligned.
  */
 enum { WQ_W8_INT8 = 0, WQ_W8_E4M3 = 1 };
 WQ_API int wq_gemm_w8a16(const void *X, int64_t M, int64_t K, const void *Wq, int w_fmt,
