@@ -114,6 +114,28 @@ def test_matches_dequantized_bf16_product():
     assert err <= REL_ROW_TOL
 
 
+def test_non_finite_activation_chunks():
+    """int8 codes at M <= 4 read X in fixed point; a chunk of X holding an
+    infinity or a NaN is multiplied in fp32 instead, so the row follows IEEE
+    arithmetic (inf * 0 = NaN) like the oracle, and the other row stays within
+    the tolerance."""
+    W = make_weight(64, 1024, 0.02, seed=4)
+    q, s, ofmt = weight_codes(W, "int8")
+    X = make_activation(3, 1024, seed=8).float()
+    X[1, 5] = float("inf")
+    X[2, 700] = float("nan")
+    X = X.to(torch.bfloat16)
+    Y = wq.gemm_w8a16(X.cuda(), q, s).float().cpu().numpy()
+    Yref, st = oracle.gemm_w8a16(bf16_bits(X), q.cpu().numpy(), ofmt, s.cpu().numpy(), 0, 64)
+    assert np.array_equal(np.isnan(Y[1:]), np.isnan(Yref[1:]))
+    assert np.array_equal(np.isinf(Y[1:]), np.isinf(Yref[1:]))
+    fin = np.isfinite(Yref[1:])
+    assert np.array_equal(np.sign(Y[1:][np.isinf(Y[1:])]), np.sign(Yref[1:][np.isinf(Yref[1:])]))
+    assert fin.sum() == 0 or np.all(np.isfinite(Y[1:][fin]))
+    err = rel_row_error(Y[:1], Yref[:1], True)
+    assert err <= REL_ROW_TOL
+
+
 def test_arguments():
     X = make_activation(2, 128, seed=1).cuda()
     q = torch.zeros((16, 128), dtype=torch.int8, device="cuda")
