@@ -109,3 +109,33 @@ def test_exact_down_to_two_to_the_minus_five_of_the_maximum():
     assert (err[np.abs(x) >= amax * 2.0 ** -5] == 0).all()
     assert (err <= amax * 2.0 ** -13).all()
     assert (err > 0).any()
+
+
+@pytest.mark.parametrize("N,K,M", [(136, 192, 1), (264, 4160, 4), (512, 4096, 2)])
+def test_w8a16_int8_fixed_point_x(N, K, M):
+    """The W8A16 decode with int8 codes reads X the same way: per activation
+    row and 128-element group, x' = rint(x 2^e) (the magic-constant rounding);
+    a lane's 16 codes times x' (two signed DP2A per code word) is an exact
+    integer below 2^24, scaled by 2^-e.  On weights with outlier rows and
+    activations with six outlier dims the product stays well inside the
+    2e-3 row bound against the fp64 oracle."""
+    W = make_weight(N, K, 0.02, seed=N + K, outlier_frac=0.02, outlier_scale=20.0).float().numpy()
+    s = np.maximum(np.abs(W).max(axis=1) / np.float32(127), np.float32(1e-8)).astype(np.float32)
+    q = np.clip(np.rint(W / s[:, None]), -127, 127).astype(np.int64)
+    X = make_activation(M, K, seed=M + K, outlier_dims=6)
+    x = X.float().numpy()
+    Y = np.zeros((M, N))
+    for g0 in range(0, K, 128):
+        xg = x[:, g0:g0 + 128]
+        xi, e = prepare(xg)
+        assert np.abs(xi).max() <= 2 ** 13                      # signed 16-bit DP2A operand
+        np.testing.assert_array_equal(magic_round(xg, e), xi)   # the kernel's rounding
+        for l0 in range(0, xg.shape[1], 16):                    # one lane's 16 codes
+            isum = xi[:, l0:l0 + 16] @ q[:, g0 + l0:g0 + l0 + 16].T
+            assert np.abs(isum).max() < 2 ** 24                 # exact in binary32
+            Y += isum * np.exp2(-e)[:, None]
+    Y *= s[None, :]
+    Yref, st = oracle.gemm_w8a16(bf16_bits(X), q.astype(np.int8), oracle.W_I8, s)
+    assert st == oracle.OK
+    err = np.abs(Y - Yref).max(axis=1) / np.linalg.norm(Yref, axis=1)
+    assert err.max() <= 5e-4, err.max()
